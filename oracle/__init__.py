@@ -1,0 +1,182 @@
+"""CPU oracle for the AWQ W4A16 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never does, and
+the oracle never imports the product: the two share nothing but the seeded
+input generators in ``synth``.
+
+The arithmetic lives in ``awq_oracle.c`` (plain scalar C, compiled with
+``-ffp-contract=off -fno-fast-math``); this module only compiles it on first
+use and marshals numpy arrays through ctypes.  Each function states the page
+and section it restates; the C file holds the step-by-step readings.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "awq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_awq.so")
+_lock = threading.Lock()
+_lib = None
+
+OK, ERR_NULL, ERR_SHAPE, ERR_NONFINITE = 0, 1, 2, 4
+GROUP = 128
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what} failed with status {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile awq_oracle.c into liboracle_awq.so next to it (gcc, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+               "-shared", "-pthread", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            lib.awq_oracle_half_to_double.argtypes = [ctypes.c_uint16]
+            lib.awq_oracle_half_to_double.restype = ctypes.c_double
+            lib.awq_oracle_double_to_half.argtypes = [ctypes.c_double]
+            lib.awq_oracle_double_to_half.restype = ctypes.c_uint16
+            lib.awq_oracle_act_stats.argtypes = [P, I64, I64, P]
+            lib.awq_oracle_compute_scales.argtypes = [P, I64, P]
+            lib.awq_oracle_quantize_pack.argtypes = [P, P, I64, I64, P, P, P]
+            lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
+            lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
+            for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
+                      lib.awq_oracle_quantize_pack, lib.awq_oracle_dequant, lib.awq_oracle_matmul):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _h(a) -> np.ndarray:
+    """binary16 data as a C-contiguous uint16 view (accepts float16 or uint16)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected float16/uint16 bits, got {a.dtype}")
+    return a
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise OracleError(code, what)
+
+
+def half_to_double(bits: int) -> float:
+    """Exact value of one binary16 bit pattern (IEEE 754 binary16 definition)."""
+    return _load().awq_oracle_half_to_double(int(bits) & 0xFFFF)
+
+
+def double_to_half(x: float) -> int:
+    """Bit pattern of the binary16 nearest to x, ties to even (one rounding)."""
+    return int(_load().awq_oracle_double_to_half(float(x)))
+
+
+def act_stats(xcal) -> np.ndarray:
+    """m[k] = mean_r |xcal[r, k]| (exact double sum, one division, float result).
+
+    Lansai AWQ explainer, "AWQ 的四步链路", row "采集激活": calibration forward,
+    per-channel input magnitude.  xcal: binary16 [R, K] -> float32 [K].
+    """
+    x = _h(xcal)
+    R, K = x.shape
+    m = np.empty(K, dtype=np.float32)
+    _check(_load().awq_oracle_act_stats(_p(x), R, K, _p(m)), "act_stats")
+    return m
+
+
+def compute_scales(m) -> np.ndarray:
+    """s = sqrt(max(m, 1e-8)) / sqrt(max t * min t), rounded once to binary16.
+
+    Lansai AWQ explainer, "AWQ 的四步链路" (Y = (X/s)(sW), s > 0 per input
+    channel); "Awq Quantization", "How AWQ Works" (objective L(s)).
+    m: float32 [K] -> float16 [K].
+    """
+    m = np.ascontiguousarray(m, dtype=np.float32)
+    s = np.empty(m.shape[0], dtype=np.uint16)
+    _check(_load().awq_oracle_compute_scales(_p(m), m.shape[0], _p(s)), "compute_scales")
+    return s.view(np.float16)
+
+
+def quantize_pack(W, s):
+    """Fold s into W, asymmetric 4-bit group-128 quantization, pack.
+
+    "Awq Quantization", "Group Size Configuration" / "Zero-Point
+    Quantization"; lansai explainer, four-step chain ("真实量化/打包").
+    W: binary16 [K, N] (Y = X W), s: binary16 [K].
+    Returns (Q int32 [K/8, N], scales float16 [K/128, N], zeros int32 [K/128, N/8]).
+    """
+    w = _h(W)
+    sv = _h(s)
+    K, N = w.shape
+    if sv.shape != (K,):
+        raise ValueError("s must have shape [K]")
+    Q = np.zeros((max(K // 8, 1), N), dtype=np.int32)
+    sc = np.zeros((max(K // GROUP, 1), N), dtype=np.uint16)
+    z = np.zeros((max(K // GROUP, 1), max(N // 8, 1)), dtype=np.int32)
+    _check(_load().awq_oracle_quantize_pack(_p(w), _p(sv), K, N, _p(Q), _p(sc), _p(z)),
+           "quantize_pack")
+    return Q, sc.view(np.float16), z
+
+
+def dequant(Q, scales, zeros) -> np.ndarray:
+    """w_hat = (q - z) * scale (the fake-quantized weights), float64 [K, N]."""
+    Q = np.ascontiguousarray(Q, dtype=np.int32)
+    sc = _h(scales)
+    z = np.ascontiguousarray(zeros, dtype=np.int32)
+    K, N = Q.shape[0] * 8, Q.shape[1]
+    out = np.empty((K, N), dtype=np.float64)
+    _check(_load().awq_oracle_dequant(_p(Q), _p(sc), _p(z), K, N, _p(out)), "dequant")
+    return out
+
+
+def matmul(X, s, Q, scales, zeros, cols=None, precision: int = 64, nthreads: int = 1) -> np.ndarray:
+    """Y = (X / s) . dequant(Q) by the plain definition, for the output columns ``cols``.
+
+    Lansai explainer, four-step chain: Y = (X/s)(sW).  precision=64 computes
+    everything in double; precision=32 is the dequantise-then-float-matmul
+    (IEEE float division for X/s, float accumulation, k ascending, no FMA).
+    X: binary16 [M, K].  Returns float64 [M, len(cols)].
+    """
+    x = _h(X)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    sv = _h(s)
+    Q = np.ascontiguousarray(Q, dtype=np.int32)
+    sc = _h(scales)
+    z = np.ascontiguousarray(zeros, dtype=np.int32)
+    M, K = x.shape
+    N = Q.shape[1]
+    if cols is None:
+        cols = np.arange(N, dtype=np.int64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    Y = np.empty((M, cols.shape[0]), dtype=np.float64)
+    _check(_load().awq_oracle_matmul(_p(x), _p(sv), _p(Q), _p(sc), _p(z), M, K, N, _p(cols),
+                                     cols.shape[0], _p(Y), int(precision), int(nthreads)),
+           "matmul")
+    return Y
