@@ -1,0 +1,501 @@
+#!/usr/bin/env python3
+"""Benchmark of the AWQ W4A16 linear layer on B200.
+
+Headline: the Mistral-7B-shaped decode set (M = 1; K x N = 4096 x 6144 QKV,
+4096 x 4096 O, 4096 x 28672 gate+up, 14336 x 4096 down).  One step is one
+decode pass through a layer: the four fused-dequantization GEMVs, each
+reading that layer's packed weights once.  Layers rotate (distinct weights,
+footprint above twice the L2 size) so the weights always come from HBM.
+The metric is packed-weight bytes (4-bit codes + binary16 steps + 4-bit zero
+points, 0.5195 B per weight) per second.
+
+Also reported on the same line: the prefill GEMM (7B shapes, M = 4096) in
+TFLOP/s, the one-off quantization pass (act_stats + compute_scales +
+quantize_pack) in GB/s of fp16 weights read, the end-to-end number through
+the public API with host buffers, and the CPU oracle timed on the host cores.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       (N > 1: launch under torch.distributed.run; each rank runs its own
+       replica of the workload, value = all ranks' bytes / max-over-ranks time)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W4A16 matmul: weight GB/s (M=1) & TFLOP/s (M>=256) vs B200 roofline"
+WORKLOAD_ID = 2
+BYTES_PER_WEIGHT = 0.5 + 2 / 128 + 0.5 / 128  # codes + steps + zero points
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantization_quantize_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+def build_layers(awq, nlayers, device, workload=WORKLOAD_ID):
+    """Quantize `nlayers` distinct synthetic layers on the GPU (kept packed)."""
+    wl = synth.WORKLOADS[workload]
+    layers = []
+    for li in range(nlayers):
+        projs = []
+        for si, (K, N, label) in enumerate(wl.shapes):
+            L = synth.make_layer(workload, li, M=1, K=K, N=N, R=wl.R, device=device, shape_id=si)
+            s = awq.compute_scales(awq.act_stats(L.Xcal))
+            Q, sc, z = awq.quantize_pack(L.W, s)
+            projs.append(dict(K=K, N=N, label=label, X=L.X, s=s, Q=Q, sc=sc, z=z,
+                              Y=torch.empty(1, N, dtype=torch.float16, device=device)))
+            del L
+        layers.append(projs)
+    torch.cuda.synchronize()
+    return layers
+
+
+def weight_bytes(K, N):
+    return K * N * BYTES_PER_WEIGHT
+
+
+def algorithmic_bytes(M, K, N):
+    return weight_bytes(K, N) + 2 * M * K + 2 * K + 2 * M * N
+
+
+def run_ours(args, rank, world, device):
+    import weight_only_quantization_quantize_b200 as awq
+    awq.lib()
+    peaks, peak_src = load_peaks()
+    L2 = torch.cuda.get_device_properties(device).L2_cache_size
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    layer_bytes = sum(weight_bytes(K, N) for K, N, _ in wl.shapes)
+    nlayers = max(2, math.ceil(2 * L2 / layer_bytes) + 1)
+    layers = build_layers(awq, nlayers, device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        for p in layers[i % nlayers]:
+            awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"])
+
+    # warm-up, then capture K steps in one CUDA graph (launch-bound decode loop)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(args.steps):
+            step(i)
+    g.replay()  # one untimed replay
+    torch.cuda.synchronize()
+
+    dist = world > 1
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The timed region lasts milliseconds, shorter than the 200 ms sampling
+    # period, so clocks are sampled over ~1 s of the same load that ends with
+    # the timed replay.
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            g.replay()
+            torch.cuda.synchronize()
+        if dist:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    del g
+
+    bytes_step = layer_bytes
+    value = world * bytes_step * args.steps / (ms * 1e-3) / 1e9
+    alg_step = sum(algorithmic_bytes(1, K, N) for K, N, _ in wl.shapes)
+    achieved = alg_step * args.steps / (ms * 1e-3) / 1e9
+    launches = 4 * args.steps
+    traffic = stored_traffic("gemv_decode_7b")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": peak_src,
+                "kernel": "small_m_kernel<1,prologue> (GEMV)",
+                "bytes_per_launch_avg": round(alg_step / 4)}
+
+    # ---- end to end through the public API: pinned host X in, host Y out, every step
+    e2e = run_e2e(awq, layers, args, device)
+
+    extra = {}
+    if not args.quick and rank == 0:
+        extra["prefill_7b_m4096"] = run_prefill(awq, device, peaks)
+        extra["quantize_7b_layer"] = run_quantize(awq, device, layers, peaks)
+        extra["small_batch_13b_m48"] = run_small_batch(awq, device, peaks)
+
+    cpu = run_cpu_baseline(rank, world) if rank == 0 else None
+    return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, launches=launches,
+                clocks=clk.summary(), extra=extra, cpu=cpu, nlayers=nlayers, L2=L2)
+
+
+def run_e2e(awq, layers, args, device):
+    stream = torch.cuda.current_stream(device)
+    nl = len(layers)
+    hx = [[torch.empty(1, p["K"], dtype=torch.float16).pin_memory() for p in layer] for layer in layers]
+    hy = [[torch.empty(1, p["N"], dtype=torch.float16).pin_memory() for p in layer] for layer in layers]
+    for li, layer in enumerate(layers):
+        for pi, p in enumerate(layer):
+            hx[li][pi].copy_(p["X"].cpu())
+    dx = [[torch.empty_like(p["X"]) for p in layer] for layer in layers]
+    h2d = sum(2 * p["K"] for p in layers[0])
+    d2h = sum(2 * p["N"] for p in layers[0])
+
+    def step(i):
+        li = i % nl
+        for pi, p in enumerate(layers[li]):
+            dx[li][pi].copy_(hx[li][pi], non_blocking=True)
+            awq.w4a16_gemv(dx[li][pi], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"])
+            hy[li][pi].copy_(p["Y"], non_blocking=True)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    wb = sum(weight_bytes(p["K"], p["N"]) for p in layers[0])
+    return {"value": round(wb * args.steps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / args.steps, 4), "path": "python binding -> C ABI, eager"}
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def run_prefill(awq, device, peaks, M=4096, reps=5):
+    """7B prefill GEMMs (tcgen05 path), TFLOP/s over the four shapes."""
+    wl = synth.WORKLOADS[4]
+    projs = []
+    for si, (K, N, label) in enumerate(wl.shapes):
+        L = synth.make_layer(4, 0, M=M, K=K, N=N, R=wl.R, device=device, shape_id=si)
+        s = awq.compute_scales(awq.act_stats(L.Xcal))
+        Q, sc, z = awq.quantize_pack(L.W, s)
+        ws = torch.empty(awq.gemm_workspace_size(M, K, N), dtype=torch.uint8, device=device)
+        projs.append(dict(K=K, N=N, X=L.X, s=s, Q=Q, sc=sc, z=z, ws=ws,
+                          Y=torch.empty(M, N, dtype=torch.float16, device=device)))
+        del L
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+
+    def step():
+        for p in projs:
+            awq.w4a16_gemm(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"], workspace=p["ws"])
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    flops = sum(2 * M * p["K"] * p["N"] for p in projs)
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {"M": M, "ms_per_layer": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak,
+            "frac": round(tf / peak, 4), "includes": "X/s pre-pass + tcgen05 GEMM, 4 shapes",
+            "l2": "256 MB buffer rewritten before each timed layer"}
+
+
+def run_small_batch(awq, device, peaks, M=48, reps=10):
+    """13B small-batch GEMMs (register-fed tensor cores), weight GB/s."""
+    wl = synth.WORKLOADS[3]
+    projs = []
+    for si, (K, N, label) in enumerate(wl.shapes):
+        L = synth.make_layer(3, 0, M=M, K=K, N=N, R=wl.R, device=device, shape_id=si)
+        s = awq.compute_scales(awq.act_stats(L.Xcal))
+        Q, sc, z = awq.quantize_pack(L.W, s)
+        ws = torch.empty(awq.gemm_workspace_size(M, K, N), dtype=torch.uint8, device=device)
+        projs.append(dict(K=K, N=N, X=L.X, s=s, Q=Q, sc=sc, z=z, ws=ws,
+                          Y=torch.empty(M, N, dtype=torch.float16, device=device)))
+        del L
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+
+    def step():
+        for p in projs:
+            awq.w4a16_gemm(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"], workspace=p["ws"])
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    wb = sum(weight_bytes(p["K"], p["N"]) for p in projs)
+    gbs = wb / (ms * 1e-3) / 1e9
+    return {"M": M, "ms_per_layer": round(ms, 4), "weight_gbs": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "includes": "X/s pre-pass + 4 GEMMs"}
+
+
+def run_quantize(awq, device, layers, peaks, reps=5):
+    """act_stats + compute_scales + quantize_pack over one 7B layer (fp16 W read once)."""
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    ins = []
+    for si, (K, N, label) in enumerate(wl.shapes):
+        L = synth.make_layer(WORKLOAD_ID, 99, M=1, K=K, N=N, R=wl.R, device=device, shape_id=si)
+        ins.append(L)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    times = []
+    for r in range(reps + 2):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for L in ins:
+            s = awq.compute_scales(awq.act_stats(L.Xcal))
+            awq.quantize_pack(L.W, s)
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 2:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    moved = sum(2 * L.K * L.N + weight_bytes(L.K, L.N) + 2 * L.R * L.K for L in ins)
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"ms_per_layer": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "bytes": "fp16 W read + packed write + calibration rows"}
+
+
+def _oracle_sample(oracle, K, N, label, si, frac, offset=0):
+    """Oracle inputs for a column sample of one projection (quantization is per column)."""
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    L = synth.make_layer(WORKLOAD_ID, 0, M=1, K=K, N=N, R=wl.R, device="cpu", shape_id=si)
+    ncols = max(8, (int(N * frac) // 8) * 8)
+    cols = (np.arange(ncols, dtype=np.int64) * (N // ncols) + offset) % N
+    s = oracle.compute_scales(oracle.act_stats(L.Xcal.numpy()))
+    Wsub = np.ascontiguousarray(L.W.numpy()[:, cols])
+    Q, sc, z = oracle.quantize_pack(Wsub, s)
+    return L.X.numpy(), s, Q, sc, z, K, ncols
+
+
+def run_cpu_baseline(rank, world, fraction=0.25):
+    """The oracle (dequantise-then-float matmul) on the host cores: a bounded sample."""
+    import oracle
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    cores = os.cpu_count() or 1
+    total_bytes, total_s = 0.0, 0.0
+    for si, (K, N, label) in enumerate(wl.shapes):
+        X, s, Q, sc, z, K, ncols = _oracle_sample(oracle, K, N, label, si, fraction)
+        t0 = time.perf_counter()
+        oracle.matmul(X, s, Q, sc, z, precision=32, nthreads=cores)
+        total_s += time.perf_counter() - t0
+        total_bytes += weight_bytes(K, ncols)
+    return {"value": round(total_bytes / total_s / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"7B decode layer, M=1, {int(fraction * 100)}% of each projection's columns "
+                      f"(all K), float dequantise-then-matmul, {cores} threads"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    if rank != 0:
+        return
+    import oracle
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    cores = os.cpu_count() or 1
+    frac = 1 / 16
+    prepared = [_oracle_sample(oracle, K, N, label, si, frac)
+                for si, (K, N, label) in enumerate(wl.shapes)]
+
+    def step(i):
+        b = 0.0
+        for X, s, Q, sc, z, K, ncols in prepared:
+            oracle.matmul(X, s, Q, sc, z, precision=32, nthreads=cores)
+            b += weight_bytes(K, ncols)
+        return b
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    tot = 0.0
+    for i in range(args.steps):
+        tot += step(i)
+    sec = time.perf_counter() - t0
+    value = tot / sec / 1e9
+    sample = (f"7B decode layer, M=1, 1/16 of each projection's columns per step (all K), "
+              f"float dequantise-then-matmul oracle, {cores} threads")
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "shapes": [list(x[:2]) for x in wl.shapes], "M": 1},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline only (no extra sections)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        r = run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    line = {
+        "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"] / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "shapes": [list(x[:2]) for x in wl.shapes], "M": 1,
+                   "layers_rotated": r["nlayers"],
+                   "l2": f"inputs larger than L2: {r['nlayers']} distinct layers rotated "
+                         f"({r['nlayers'] * 113.3:.0f} MB of packed weights > 2 x {r['L2'] / 2**20:.0f} MiB L2)",
+                   "parallelism": f"replicas x{world}", "timing": "CUDA graph of all timed steps, CUDA events",
+                   "clocks_window": "nvidia-smi every 200 ms over ~1 s of identical load ending with the timed replay"},
+        "roofline": r["roofline"], "cpu_baseline": r["cpu"], "e2e": r["e2e"],
+        "gpu_launches": r["launches"], "clocks": r["clocks"],
+    }
+    line.update(r["extra"])
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * awq_b200.h -- C ABI of libawq_b200.so, the AWQ W4A16 group-quantized linear
+ * layer for NVIDIA B200 (sm_100a).
+ *
+ * The operations restate the activation-aware weight quantization described
+ * on the AWQ pages:
+ *   - lansai AWQ explainer (ai.lansai.wang/107648), section "AWQ 的四步链路":
+ *     Y = XW is rewritten with a positive per-input-channel scale s as
+ *     Y = (X/s)(sW); calibration activations give per-channel magnitudes;
+ *     the scaled weights are quantized by group and packed with their
+ *     scale and zero point;
+ *   - "Awq Quantization" (skillselion.com), "How AWQ Works" (objective
+ *     ||Q(W*s)(s^-1*X) - W*X||), "Group Size Configuration" (groups of 128,
+ *     4 bits), "Zero-Point Quantization" (asymmetric codes with an offset),
+ *     "WQLinear Kernel Variants" (a GEMV kernel for single-token decode and
+ *     a GEMM kernel for batches).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE memory owned by the caller, on the
+ *     current CUDA device; the library allocates nothing on these calls and
+ *     keeps no pointer after it returns.
+ *   - float16 data are passed as IEEE binary16 bit patterns (uint16_t).
+ *   - Every tensor is dense row-major; device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on that stream.
+ *   - Errors detectable on the host (null pointers, shapes, alignment,
+ *     device architecture, workspace size) are returned before anything is
+ *     launched.  Errors found on the device (non-finite inputs, a bounded wait
+ *     that ran out) are written as an awq_status_t value into *dev_status if
+ *     dev_status is not NULL; the first error wins, the library never clears
+ *     it: the caller zeroes it and reads it after synchronizing the stream.
+ *   - Outputs must not alias inputs.
+ *
+ * Data layout (K input channels, N output channels, G = K/128 groups)
+ *   W       binary16 [K, N]     Y = X W
+ *   s       binary16 [K]        per-input-channel scale
+ *   Q       int32 [K/8, N]      bits [4j, 4j+4) of Q[k8, n] hold the 4-bit code
+ *                               of row 8*k8 + j, column n (sequential nibbles)
+ *   scales  binary16 [G, N]     per-group step of the 4-bit grid
+ *   zeros   int32 [G, N/8]      bits [4j, 4j+4) of zeros[g, n8] hold the zero
+ *                               point of column 8*n8 + j
+ *   X       binary16 [M, K]     activations;  Y binary16 [M, N]
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+#define AWQ_GROUP_SIZE 128      /* q_group_size ("Group Size Configuration") */
+#define AWQ_W_BIT 4             /* w_bit: codes 0..15                          */
+#define AWQ_MAX_CALIB_ROWS 8192 /* keeps the double sum of |x| exact           */
+#define AWQ_MAX_K 262144
+#define AWQ_MAX_N 1048576
+#define AWQ_MAX_M 1048576
+#define AWQ_ABI_VERSION 1
+
+typedef enum {
+    AWQ_OK = 0,
+    AWQ_ERR_NULL = 1,           /* a required pointer is NULL                      */
+    AWQ_ERR_SHAPE = 2,          /* K % 128, N % 8, M < 1, R < 1, or above a limit  */
+    AWQ_ERR_ALIGN = 3,          /* a device pointer is not 16-byte aligned         */
+    AWQ_ERR_NONFINITE = 4,      /* NaN/Inf in W, s, X_cal or the statistics        */
+    AWQ_ERR_ARCH = 5,           /* the current device is not sm_100 (B200)         */
+    AWQ_ERR_CUDA = 6,           /* a CUDA runtime/driver call or launch failed     */
+    AWQ_ERR_DEVICE_TIMEOUT = 7, /* a bounded wait inside a kernel ran out          */
+    AWQ_ERR_WORKSPACE = 8       /* workspace NULL or smaller than required         */
+} awq_status_t;
+
+typedef void *awq_stream_t; /* a cudaStream_t */
+
+/* Human-readable name of a status code (static storage). */
+AWQ_API const char *awq_status_string(awq_status_t status);
+
+/* AWQ_ABI_VERSION of the loaded library. */
+AWQ_API int awq_abi_version(void);
+
+/*
+ * Activation statistics -- lansai explainer, "AWQ 的四步链路", row "采集激活"
+ * (collect the layer-input magnitude on calibration data).
+ *   m[k] = (1/R) * sum_r |xcal[r, k]|
+ * The sum is exact (double; every binary16 is a multiple of 2^-24), divided
+ * once in double and rounded once to float, so the result does not depend on
+ * the reduction order.
+ *   xcal  binary16 [R, K], 1 <= R <= AWQ_MAX_CALIB_ROWS ("Calibration samples
+ *         are empty" is AWQ_ERR_SHAPE), K % 8 == 0
+ *   m     float [K] (output)
+ * Device errors: AWQ_ERR_NONFINITE if xcal holds NaN/Inf (m is still written).
+ */
+AWQ_API awq_status_t awq_act_stats(const uint16_t *xcal, int64_t R, int64_t K, float *m,
+                           int32_t *dev_status, awq_stream_t stream);
+
+/*
+ * Per-channel scale -- lansai explainer, "AWQ 的四步链路" (Y = (X/s)(sW));
+ * "Awq Quantization", "How AWQ Works" (s lowers ||Q(W*s)(s^-1*X) - W*X||).
+ * One point of the scale family: s = m^0.5, normalised by the geometric
+ * centre of its extremes:
+ *   t_k = sqrt(max(m_k, 1e-8)),  c = sqrt(max_j t_j * min_j t_j),
+ *   s_k = binary16_RNE(t_k / c)          (double arithmetic, IEEE rounding)
+ *   m  float [K] (K >= 1);  s  binary16 [K] (output)
+ * Device errors: AWQ_ERR_NONFINITE if some m_k is NaN/Inf/negative (s is
+ * then left unspecified).
+ */
+AWQ_API awq_status_t awq_compute_scales(const float *m, int64_t K, uint16_t *s, int32_t *dev_status,
+                                awq_stream_t stream);
+
+/*
+ * Fold, quantize and pack -- lansai explainer, "AWQ 的四步链路" (enlarge the
+ * salient channels' weights, sW, then quantize by group; row "真实量化/打包");
+ * "Awq Quantization", "Group Size Configuration", "Zero-Point Quantization".
+ * Per group g (rows 128g..128g+127) and column n, with w' = float(w) * float(s_k):
+ *   r       = max(max w' - min w', 1e-5f)
+ *   scale_h = binary16_RNE(r / 15)  (the smallest subnormal if that is 0)
+ *   z       = clamp(rint(-min w' / scale_h), 0, 15)
+ *   q       = clamp(rint(w' / scale_h) + z, 0, 15)   (rint: ties to even)
+ * all in IEEE float arithmetic; the outputs are bit-exact functions of W, s.
+ *   W binary16 [K, N], s binary16 [K] (> 0), K % 128 == 0, N % 8 == 0
+ *   Q int32 [K/8, N], scales binary16 [K/128, N], zeros int32 [K/128, N/8] (outputs)
+ * Device errors: AWQ_ERR_NONFINITE if W or s holds NaN/Inf or s <= 0
+ * ("NaN detected in weights", "Awq Quantization", Troubleshooting Guide).
+ */
+AWQ_API awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                               int32_t *Q, uint16_t *scales, int32_t *zeros,
+                               int32_t *dev_status, awq_stream_t stream);
+
+/*
+ * Fused-dequantization matmul -- lansai explainer, "AWQ 的四步链路"
+ * (Y = (X/s)(sW)); "Awq Quantization", "WQLinear Kernel Variants" (GEMV for
+ * batch size 1, GEMM for batches).
+ *   Y[m, n] = sum_k (X[m, k] / s_k) * (q[k, n] - z[g(k), n]) * scale_h[g(k), n]
+ * with the nibble unpack and (q - z) * scale dequantisation done inside the
+ * kernel (no dequantised weight matrix is ever written to memory), X / s
+ * rounded to binary16 for the tensor cores, float accumulation, Y rounded to
+ * binary16.  Results agree with the exact definition within
+ * max|dY| <= 1e-2 * max|Y| and ||dY||_F <= 5e-3 * ||Y||_F.
+ *
+ * awq_w4a16_gemv is the M = 1 (single-token decode) entry point:
+ *   X binary16 [1, K], Y binary16 [1, N].
+ * awq_w4a16_gemm takes any 1 <= M <= AWQ_MAX_M and picks its tile path
+ * internally (register-fed tensor cores for M < 64, tcgen05/TMEM for M >= 64).
+ *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack.
+ * Workspace: caller-owned device memory of at least *_workspace_size() bytes
+ * (may be NULL when that size is 0); it holds X / s and is overwritten.
+ * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
+ * (Y is then unspecified).
+ */
+AWQ_API size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N);
+AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                            const uint16_t *scales, const int32_t *zeros, int64_t K, int64_t N,
+                            uint16_t *Y, void *workspace, size_t workspace_bytes,
+                            int32_t *dev_status, awq_stream_t stream);
+
+AWQ_API size_t awq_w4a16_gemm_workspace_size(int64_t M, int64_t K, int64_t N);
+AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                            const uint16_t *scales, const int32_t *zeros, int64_t M, int64_t K,
+                            int64_t N, uint16_t *Y, void *workspace, size_t workspace_bytes,
+                            int32_t *dev_status, awq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

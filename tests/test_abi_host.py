@@ -1,0 +1,108 @@
+"""Host-side tests of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the device.
+
+Every call here fails validation on the host (null pointer, shape, alignment
+or workspace), so no kernel is launched and no GPU is needed.  The fake device
+addresses are never dereferenced.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import weight_only_quantization_quantize_b200 as awq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq_b200.h")
+
+A = 0x7F0000000000           # a 16-byte aligned fake device address
+MIS = A + 2                  # misaligned
+P = ctypes.c_void_p
+
+
+@pytest.fixture(scope="module")
+def L():
+    from weight_only_quantization_quantize_b200 import _build
+    _build.build()
+    return awq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(awq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(awq.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", awq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (awq_\w+)", out))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(L, f)
+    # nothing but the ABI is exported with the awq_ prefix
+    assert exported == set(declared_functions())
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.awq_abi_version() == 1
+    for code, name in awq.STATUS.items():
+        assert awq.status_string(code).startswith(name)
+    assert awq.status_string(99) == "AWQ_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(L):
+    assert L.awq_w4a16_gemv_workspace_size(4096, 4096) == 0
+    assert L.awq_w4a16_gemm_workspace_size(1, 4096, 4096) == 0
+    assert L.awq_w4a16_gemm_workspace_size(48, 5120, 5120) >= 2 * 48 * 5120
+    assert L.awq_w4a16_gemm_workspace_size(4096, 14336, 4096) >= 2 * 4096 * 14336
+    assert L.awq_w4a16_gemm_workspace_size(4, 100, 4096) == 0          # invalid shape
+
+
+def gemm(L, X=A, s=A, Q=A, sc=A, z=A, M=64, K=4096, N=4096, Y=A, ws=A, wsb=1 << 40, st=None):
+    return L.awq_w4a16_gemm(P(X), P(s), P(Q), P(sc), P(z), M, K, N, P(Y), P(ws), wsb, P(st), None)
+
+
+def test_matmul_validation(L):
+    assert gemm(L, X=0) == awq.ERR_NULL
+    assert gemm(L, z=0) == awq.ERR_NULL
+    assert gemm(L, Y=0) == awq.ERR_NULL
+    assert gemm(L, K=100) == awq.ERR_SHAPE            # K % 128
+    assert gemm(L, K=0) == awq.ERR_SHAPE
+    assert gemm(L, N=12) == awq.ERR_SHAPE             # N % 8
+    assert gemm(L, M=0) == awq.ERR_SHAPE
+    assert gemm(L, M=-3) == awq.ERR_SHAPE
+    assert gemm(L, K=1 << 20) == awq.ERR_SHAPE        # above AWQ_MAX_K
+    assert gemm(L, X=MIS) == awq.ERR_ALIGN
+    assert gemm(L, Q=A + 4) == awq.ERR_ALIGN
+    assert gemm(L, st=A + 1) == awq.ERR_ALIGN         # status word alignment
+    assert gemm(L, ws=0) == awq.ERR_WORKSPACE
+    assert gemm(L, wsb=100) == awq.ERR_WORKSPACE
+    r = L.awq_w4a16_gemv(P(A), P(A), P(A), P(A), P(A), 4096, 4097, P(A), None, 0, None, None)
+    assert r == awq.ERR_SHAPE
+    r = L.awq_w4a16_gemv(P(A), P(0), P(A), P(A), P(A), 4096, 4096, P(A), None, 0, None, None)
+    assert r == awq.ERR_NULL
+
+
+def test_quantize_and_stats_validation(L):
+    q = L.awq_quantize_pack
+    assert q(P(0), P(A), 128, 8, P(A), P(A), P(A), None, None) == awq.ERR_NULL
+    assert q(P(A), P(A), 192, 8, P(A), P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert q(P(A), P(A), 128, 4, P(A), P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert q(P(A), P(MIS), 128, 8, P(A), P(A), P(A), None, None) == awq.ERR_ALIGN
+    st = L.awq_act_stats
+    assert st(P(A), 0, 1024, P(A), None, None) == awq.ERR_SHAPE       # empty calibration
+    assert st(P(A), 8193, 1024, P(A), None, None) == awq.ERR_SHAPE    # exactness limit
+    assert st(P(A), 16, 1020, P(A), None, None) == awq.ERR_SHAPE
+    assert st(P(0), 16, 1024, P(A), None, None) == awq.ERR_NULL
+    assert st(P(A), 16, 1024, P(MIS), None, None) == awq.ERR_ALIGN
+    cs = L.awq_compute_scales
+    assert cs(P(A), 0, P(A), None, None) == awq.ERR_SHAPE
+    assert cs(P(A), 16, P(0), None, None) == awq.ERR_NULL

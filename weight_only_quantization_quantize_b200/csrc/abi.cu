@@ -1,0 +1,258 @@
+// abi.cu -- the extern "C" boundary of libawq_b200.so (declared in awq_b200.h).
+//
+// Host-side work only: argument validation (returned before any launch), a
+// one-time per-device architecture check, TMA descriptor encoding, workspace
+// accounting and the choice of tile path.  Every step of the computation runs
+// in the kernels of quantize.cu, matmul_small.cu and matmul_tc.cu.
+#include <mutex>
+
+#include "awq_kernels.cuh"
+
+namespace {
+
+using awq::kGroup;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+    bool checked = false;
+    bool supported = false;
+    int sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+DeviceState g_devices[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+awq_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Checks (once per device) that the current device is an sm_100 part and
+// prepares the kernels' shared-memory limits and the TMA encoder.
+awq_status_t device_ready(int *sms)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return AWQ_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_ARCH;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &d = g_devices[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, count = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return AWQ_ERR_CUDA;
+        }
+        d.supported = (major == 10 && minor == 0);
+        d.sms = count;
+        if (d.supported) {
+            if (!g_encode) {
+                void *fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                        cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || fn == nullptr) {
+                    cudaGetLastError();
+                    return AWQ_ERR_CUDA;
+                }
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+            }
+            if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess) {
+                cudaGetLastError();
+                return AWQ_ERR_CUDA;
+            }
+        }
+        d.checked = true;
+    }
+    if (!d.supported) return AWQ_ERR_ARCH;
+    *sms = d.sms;
+    return AWQ_OK;
+}
+
+// 2-D tiled tensor map over a row-major [outer, inner] array.
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle)
+{
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t elem[2] = {1, 1};
+    return g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, elem,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool matmul_shape_ok(int64_t M, int64_t K, int64_t N)
+{
+    return M >= 1 && M <= AWQ_MAX_M && K >= kGroup && K % kGroup == 0 && K <= AWQ_MAX_K && N >= 8 &&
+           N % 8 == 0 && N <= AWQ_MAX_N;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// X / s (binary16, pair-permuted) lives in the workspace unless the
+// small-batch kernel computes it in shared memory itself (M = 1 always does).
+size_t workspace_bytes(int64_t M, int64_t K) { return M == 1 ? 0 : round_up(static_cast<size_t>(2 * M * K), 256); }
+
+awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                        const uint16_t *scales, const int32_t *zeros, int64_t M, int64_t K,
+                        int64_t N, uint16_t *Y, void *ws, size_t ws_bytes, int32_t *dev_status,
+                        awq_stream_t stream)
+{
+    if (!X || !s || !Q || !scales || !zeros || !Y) return AWQ_ERR_NULL;
+    if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
+        !aligned16(Y) || (ws && !aligned16(ws)) || (dev_status && !aligned4(dev_status)))
+        return AWQ_ERR_ALIGN;
+    const size_t need = workspace_bytes(M, K);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return AWQ_ERR_WORKSPACE;
+    int sms = 0;
+    awq_status_t e = device_ready(&sms);
+    if (e != AWQ_OK) return e;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int m = static_cast<int>(M), k = static_cast<int>(K), n = static_cast<int>(N);
+    const __half *hX = reinterpret_cast<const __half *>(X);
+    const __half *hs = reinterpret_cast<const __half *>(s);
+    const __half *hsc = reinterpret_cast<const __half *>(scales);
+    __half *hY = reinterpret_cast<__half *>(Y);
+    __half *Xp = reinterpret_cast<__half *>(ws);
+
+    CUtensorMap tmQ, tmX;
+    if (M < 64) {
+        const awq::SmallMPlan plan = awq::plan_small_m(m, k, n, sms);
+        if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return AWQ_ERR_CUDA;
+        if (!plan.prologue) {
+            if (!Xp) return AWQ_ERR_WORKSPACE;
+            if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
+                           static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
+                return AWQ_ERR_CUDA;
+            e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
+            if (e != AWQ_OK) return e;
+        } else {
+            tmX = tmQ;  // unused by the kernel
+        }
+        return from_cuda(awq::launch_small_m(plan, tmQ, tmX, hX, hs, hsc, zeros, hY, m, k, n,
+                                             dev_status, st));
+    }
+    const awq::TcPlan plan = awq::plan_tc(m, k, n, sms);
+    if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 256, 8,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return AWQ_ERR_CUDA;
+    e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
+    if (e != AWQ_OK) return e;
+    return from_cuda(awq::launch_tc(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *awq_status_string(awq_status_t status)
+{
+    switch (status) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_NULL: return "AWQ_ERR_NULL: a required pointer is NULL";
+    case AWQ_ERR_SHAPE: return "AWQ_ERR_SHAPE: unsupported shape";
+    case AWQ_ERR_ALIGN: return "AWQ_ERR_ALIGN: device pointer not 16-byte aligned";
+    case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: NaN or Inf in the input";
+    case AWQ_ERR_ARCH: return "AWQ_ERR_ARCH: device is not sm_100 (B200)";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA call or launch failed";
+    case AWQ_ERR_DEVICE_TIMEOUT: return "AWQ_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
+    case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "AWQ_ERR_UNKNOWN";
+}
+
+int awq_abi_version(void) { return AWQ_ABI_VERSION; }
+
+awq_status_t awq_act_stats(const uint16_t *xcal, int64_t R, int64_t K, float *m,
+                           int32_t *dev_status, awq_stream_t stream)
+{
+    if (!xcal || !m) return AWQ_ERR_NULL;
+    if (R < 1 || R > AWQ_MAX_CALIB_ROWS || K < 8 || K % 8 != 0 || K > AWQ_MAX_K) return AWQ_ERR_SHAPE;
+    if (!aligned16(xcal) || !aligned16(m) || (dev_status && !aligned4(dev_status))) return AWQ_ERR_ALIGN;
+    int sms = 0;
+    awq_status_t e = device_ready(&sms);
+    if (e != AWQ_OK) return e;
+    return from_cuda(awq::launch_act_stats(reinterpret_cast<const __half *>(xcal), static_cast<int>(R),
+                                           static_cast<int>(K), m, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+awq_status_t awq_compute_scales(const float *m, int64_t K, uint16_t *s, int32_t *dev_status,
+                                awq_stream_t stream)
+{
+    if (!m || !s) return AWQ_ERR_NULL;
+    if (K < 1 || K > AWQ_MAX_K) return AWQ_ERR_SHAPE;
+    if (!aligned16(m) || !aligned16(s) || (dev_status && !aligned4(dev_status))) return AWQ_ERR_ALIGN;
+    int sms = 0;
+    awq_status_t e = device_ready(&sms);
+    if (e != AWQ_OK) return e;
+    return from_cuda(awq::launch_compute_scales(m, static_cast<int>(K), s, dev_status,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                               int32_t *Q, uint16_t *scales, int32_t *zeros, int32_t *dev_status,
+                               awq_stream_t stream)
+{
+    if (!W || !s || !Q || !scales || !zeros) return AWQ_ERR_NULL;
+    if (K < kGroup || K % kGroup != 0 || K > AWQ_MAX_K || N < 8 || N % 8 != 0 || N > AWQ_MAX_N)
+        return AWQ_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
+        (dev_status && !aligned4(dev_status)))
+        return AWQ_ERR_ALIGN;
+    int sms = 0;
+    awq_status_t e = device_ready(&sms);
+    if (e != AWQ_OK) return e;
+    return from_cuda(awq::launch_quantize_pack(
+        reinterpret_cast<const __half *>(W), reinterpret_cast<const __half *>(s), static_cast<int>(K),
+        static_cast<int>(N), Q, reinterpret_cast<__half *>(scales), zeros, dev_status,
+        static_cast<cudaStream_t>(stream)));
+}
+
+size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N)
+{
+    return matmul_shape_ok(1, K, N) ? workspace_bytes(1, K) : 0;
+}
+
+awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                            const uint16_t *scales, const int32_t *zeros, int64_t K, int64_t N,
+                            uint16_t *Y, void *workspace, size_t workspace_bytes_, int32_t *dev_status,
+                            awq_stream_t stream)
+{
+    return run_matmul(X, s, Q, scales, zeros, 1, K, N, Y, workspace, workspace_bytes_, dev_status,
+                      stream);
+}
+
+size_t awq_w4a16_gemm_workspace_size(int64_t M, int64_t K, int64_t N)
+{
+    return matmul_shape_ok(M, K, N) ? workspace_bytes(M, K) : 0;
+}
+
+awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                            const uint16_t *scales, const int32_t *zeros, int64_t M, int64_t K,
+                            int64_t N, uint16_t *Y, void *workspace, size_t workspace_bytes_,
+                            int32_t *dev_status, awq_stream_t stream)
+{
+    return run_matmul(X, s, Q, scales, zeros, M, K, N, Y, workspace, workspace_bytes_, dev_status,
+                      stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,226 @@
+// awq_common.cuh -- device helpers shared by the AWQ W4A16 kernels (sm_100a).
+//
+// Thin inline-PTX wrappers: mbarriers with bounded waits, TMA tile loads,
+// cp.async with mbarrier completion, warp-level tensor-core MMA, cluster
+// (distributed shared memory) access and the device status word.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "awq_b200.h"
+
+namespace awq {
+
+constexpr int kGroup = 128;
+
+// Every wait inside a kernel is bounded by wall time (%globaltimer, ns).  A
+// wait that runs out records AWQ_ERR_DEVICE_TIMEOUT and returns false; the
+// caller then skips its remaining work but still reaches every block- and
+// cluster-wide barrier, so the context survives and the host can read the
+// status word.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ void report(int32_t *status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((i & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+// ---------------------------------------------------------------- TMA
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 2-D tiled bulk-tensor load into this CTA's shared memory; completion is
+// signalled as transaction bytes on `bar`.  x is the innermost coordinate.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uint64_t *bar, int x,
+                                            int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// ---------------------------------------------------------------- cp.async
+// src_bytes == 0 zero-fills the destination without reading global memory.
+__device__ __forceinline__ void cp_async_4(void *dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// Arrive on `bar` once this thread's earlier cp.async copies have landed.
+// The arrival is counted in the barrier's initial count (.noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// ---------------------------------------------------------------- shared loads
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// ---------------------------------------------------------------- named barriers
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- cluster / DSMEM
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------- tensor cores (warp MMA)
+// D = A * B + C, A 16x16 f16 (row), B 16x8 f16 (col), C/D 16x8 f32.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- 4-bit unpack
+// One packed word holds 8 consecutive-k codes of one column (nibble j = row
+// 8*k8 + j).  OR-ing a nibble into the mantissa of binary16 1024.0 (0x6400)
+// yields exactly 1024 + q (or 1024 + 16 q for the odd nibbles); subtracting
+// 1024 + z (or scaling by 1/16 and subtracting 64 + z) leaves q - z exactly.
+// Output pairs (low, high half): d[0] = (q0, q4), d[1] = (q1, q5),
+// d[2] = (q2, q6), d[3] = (q3, q7), each minus z.
+__device__ __forceinline__ void unpack_minus_zero(uint32_t w, uint32_t za, uint32_t zb,
+                                                  uint32_t (&d)[4])
+{
+    const uint32_t w8 = w >> 8;
+    const uint32_t v0 = (w & 0x000F000Fu) | 0x64006400u;
+    const uint32_t v1 = (w & 0x00F000F0u) | 0x64006400u;
+    const uint32_t v2 = (w8 & 0x000F000Fu) | 0x64006400u;
+    const uint32_t v3 = (w8 & 0x00F000F0u) | 0x64006400u;
+    const uint32_t sixteenth = 0x2C002C00u;  // (1/16, 1/16)
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d[0]) : "r"(v0), "r"(za));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d[1]) : "r"(v1), "r"(sixteenth), "r"(zb));
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d[2]) : "r"(v2), "r"(za));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d[3]) : "r"(v3), "r"(sixteenth), "r"(zb));
+}
+
+// (-(1024 + z), -(1024 + z)) and (-(64 + z), -(64 + z)) as f16x2 bit patterns.
+__device__ __forceinline__ void zero_constants(uint32_t z, uint32_t &za, uint32_t &zb)
+{
+    // -(1024 + z): sign | exponent of 1024 | mantissa z
+    const uint32_t a = 0xE400u | z;
+    // -(64 + z) = -(1 + z/64) * 2^6: exponent 6+15 = 21 (0x5400), mantissa z*16
+    const uint32_t b = 0xD400u | (z << 4);
+    za = a | (a << 16);
+    zb = b | (b << 16);
+}
+
+}  // namespace awq

@@ -1,0 +1,46 @@
+// awq_kernels.cuh -- kernel launchers of libawq_b200 (internal, C++ only).
+#pragma once
+
+#include "awq_common.cuh"
+
+namespace awq {
+
+// quantize.cu
+cudaError_t launch_act_stats(const __half *xcal, int R, int K, float *m, int32_t *status,
+                             cudaStream_t st);
+cudaError_t launch_compute_scales(const float *m, int K, uint16_t *s, int32_t *status,
+                                  cudaStream_t st);
+cudaError_t launch_quantize_pack(const __half *W, const __half *s, int K, int N, int32_t *Q,
+                                 __half *scales, int32_t *zeros, int32_t *status,
+                                 cudaStream_t st);
+
+// matmul_small.cu -- M < 64: register-fed tensor cores, TMA weight stream
+struct SmallMPlan {
+    int mt;          // token tiles of 8
+    bool prologue;   // X / s computed inside the kernel (no workspace)
+    int splits;      // CTAs per cluster along K
+    int n_tiles;     // 128-column tiles
+    int stages;
+    size_t smem;     // dynamic shared memory bytes
+};
+SmallMPlan plan_small_m(int M, int K, int N, int num_sms);
+cudaError_t configure_small_m();
+cudaError_t launch_prescale(const __half *X, const __half *s, int M, int K, __half *Xp,
+                            cudaStream_t st);
+cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const CUtensorMap &tmX,
+                           const __half *X, const __half *s, const __half *scales,
+                           const int32_t *zeros, __half *Y, int M, int K, int N,
+                           int32_t *status, cudaStream_t st);
+
+// matmul_tc.cu -- M >= 64: tcgen05 / TMEM
+struct TcPlan {
+    int m_tiles, n_tiles;
+    size_t smem;
+};
+TcPlan plan_tc(int M, int K, int N, int num_sms);
+cudaError_t configure_tc();
+cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensorMap &tmQ,
+                      const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                      int32_t *status, cudaStream_t st);
+
+}  // namespace awq

@@ -1,0 +1,325 @@
+// matmul_tc.cu -- Y = (X / s) . dequant(Q) for M >= 64 tokens (batched and
+// prefill), the tensor-bound regime of the W4A16 linear layer, on the
+// 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Sources: lansai AWQ explainer (ai.lansai.wang/107648), "AWQ 的四步链路"
+// (Y = (X/s)(sW)); "Awq Quantization" (skillselion.com), "WQLinear Kernel
+// Variants" (GEMM kernel for batch sizes > 1), "Group Size Configuration",
+// "Zero-Point Quantization".
+//
+// One CTA computes a 128 (tokens) x 256 (output columns) tile of Y:
+//   warp 0      TMA producer: X' tile [128 x 64] (128-byte swizzled, the
+//               canonical K-major operand layout) and the packed-word tile
+//               [8 x 256]; cp.async for the group's scales and zero points.
+//   warp 1      allocates 256 TMEM columns; one lane issues
+//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) x 4
+//               per 64-k stage and commits each stage back to the producer.
+//   warps 2..5  dequantize: word -> 8 binary16 (q - z) * step values, stored
+//               as one 16-byte chunk of the K-major, 128-byte-swizzled B
+//               operand; then, after the last stage, drain TMEM (tcgen05.ld)
+//               to binary16 Y.
+// Within each 8-channel chunk the contraction runs in the pair order
+// (0,4),(1,5),(2,6),(3,7) on both operands (X' is stored that way by the
+// pre-pass), which leaves the sum unchanged.
+#include "awq_kernels.cuh"
+
+namespace awq {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;      // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;      // 32 KB
+constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 8 KB
+constexpr int kMetaBytes = 1024;            // 512 B steps + 128 B zero words, padded
+constexpr int kStageBytes = kABytes + kBBytes + kQBytes + kMetaBytes;
+constexpr int kTmemCols = 256;
+
+struct Params {
+    const __half *scales;
+    const int32_t *zeros;
+    __half *Y;
+    int32_t *status;
+    int M, K, N;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// Shared-memory operand descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), leading byte offset unused (1),
+// descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor: kind::f16, A = B = f16, D = f32, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kBM >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b)
+{
+    return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(a))) |
+           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(b))) << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
+              const Params p)
+{
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *smem = align1024(smem_dyn);
+    uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    uint64_t *full_b = full_load + kStages;
+    uint64_t *empty = full_b + kStages;
+    uint64_t *tmem_full = empty + kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tmem_full + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kBN;
+    const int m0 = blockIdx.y * kBM;
+    const int KB = p.K / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full_load[i], 1 + 32);
+            mbar_init(&full_b[i], 4);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(tmem_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            prefetch_tmap(&tmQ);
+        }
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int st = kb % kStages;
+            if (kb >= kStages && !mbar_wait(&empty[st], ((kb / kStages) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t *stg = smem + st * kStageBytes;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full_load[st], kABytes + kQBytes);
+                tma_load_2d(stg, &tmA, &full_load[st], kb * kBK, m0);
+                tma_load_2d(stg + kABytes + kBBytes, &tmQ, &full_load[st], n0, kb * (kBK / 8));
+            }
+            uint8_t *meta = stg + kABytes + kBBytes + kQBytes;
+            const int g = (kb * kBK) / kGroup;
+            const int n = n0 + 8 * lane;
+            const bool in_s = n < p.N;
+            cp_async_16(meta + 16 * lane, p.scales + static_cast<size_t>(g) * p.N + (in_s ? n : 0),
+                        in_s ? 16u : 0u);
+            const int wi = n0 / 8 + lane;
+            const bool in_z = wi < p.N / 8;
+            cp_async_4(meta + 512 + 4 * lane,
+                       p.zeros + static_cast<size_t>(g) * (p.N / 8) + (in_z ? wi : 0), in_z ? 4u : 0u);
+            cp_async_arrive_noinc(&full_load[st]);
+        }
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int st = kb % kStages;
+            const uint32_t par = (kb / kStages) & 1;
+            if (!mbar_wait(&full_load[st], par) || !mbar_wait(&full_b[st], par)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t a0 = smem_u32(smem + st * kStageBytes);
+                const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    tc_mma(tmem_base, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k),
+                           (kb > 0 || k > 0) ? 1u : 0u);
+                tc_commit(&empty[st]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            if (ok)
+                tc_commit(tmem_full);
+            else
+                report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ dequant
+        const int tid = threadIdx.x - 64;  // 0..127
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int st = kb % kStages;
+            if (!mbar_wait(&full_load[st], (kb / kStages) & 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t *stg = smem + st * kStageBytes;
+            const uint8_t *q = stg + kABytes + kBBytes;
+            const uint8_t *meta = q + kQBytes;
+            const uint32_t bbase = smem_u32(stg + kABytes);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int n = tid + 128 * half;
+                const uint16_t sbits = reinterpret_cast<const uint16_t *>(meta)[n];
+                const uint32_t sc2 = static_cast<uint32_t>(sbits) | (static_cast<uint32_t>(sbits) << 16);
+                const uint32_t zw = reinterpret_cast<const uint32_t *>(meta + 512)[n >> 3];
+                uint32_t za, zb;
+                zero_constants((zw >> (4 * (n & 7))) & 15u, za, zb);
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const uint32_t w = reinterpret_cast<const uint32_t *>(q + r * (kBN * 4))[n];
+                    uint32_t d[4];
+                    unpack_minus_zero(w, za, zb, d);
+                    uint32_t o[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(d[i]), "r"(sc2));
+                    const uint32_t dst = bbase + n * 128 + ((r ^ (n & 7)) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]),
+                                 "r"(o[1]), "r"(o[2]), "r"(o[3])
+                                 : "memory");
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_b[st]);
+        }
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+
+        // ------------------------------------------------------------ epilogue
+        if (ok && mbar_wait(tmem_full, 0)) {
+            tc_fence_after();
+            const int quarter = warp & 3;  // TMEM lanes this warp may access
+            const int row = quarter * 32 + lane;
+            const int m = m0 + row;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kBN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + c0, v);
+                if (m < p.M) {
+                    __half *dst = p.Y + static_cast<size_t>(m) * p.N + n0 + c0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (n0 + c0 + 8 * i < p.N) {
+                            uint4 o;
+                            o.x = pack_half2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                            o.y = pack_half2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                            o.z = pack_half2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                            o.w = pack_half2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                            *reinterpret_cast<uint4 *>(dst + 8 * i) = o;
+                        }
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+TcPlan plan_tc(int M, int K, int N, int num_sms)
+{
+    (void)K;
+    (void)num_sms;
+    TcPlan pl{};
+    pl.m_tiles = (M + kBM - 1) / kBM;
+    pl.n_tiles = (N + kBN - 1) / kBN;
+    pl.smem = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+    return pl;
+}
+
+cudaError_t configure_tc()
+{
+    return cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(plan_tc(128, 128, 256, 1).smem));
+}
+
+cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensorMap &tmQ,
+                      const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                      int32_t *status, cudaStream_t st)
+{
+    Params prm{scales, zeros, Y, status, M, K, N};
+    dim3 grid(plan.n_tiles, plan.m_tiles);
+    tc_kernel<<<grid, kThreads, plan.smem, st>>>(tmA, tmQ, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace awq
