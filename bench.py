@@ -444,6 +444,30 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(workload, M, reps):
+    """One synthetic layer of `workload`, each projection called `reps` times (for ncu)."""
+    import weight_only_quantization_quantize_b200 as awq
+    torch.cuda.set_device(0)
+    wl = synth.WORKLOADS[workload]
+    projs = []
+    for si, (K, N, label) in enumerate(wl.shapes):
+        L = synth.make_layer(workload, 0, M=M, K=K, N=N, R=wl.R, device="cuda", shape_id=si)
+        s = awq.compute_scales(awq.act_stats(L.Xcal))
+        Q, sc, z = awq.quantize_pack(L.W, s)
+        ws = torch.empty(max(awq.gemm_workspace_size(M, K, N), 16), dtype=torch.uint8, device="cuda")
+        projs.append((L.X, s, Q, sc, z, ws))
+        del L
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        for X, s, Q, sc, z, ws in projs:
+            if M == 1:
+                awq.w4a16_gemv(X, s, Q, sc, z)
+            else:
+                awq.w4a16_gemm(X, s, Q, sc, z, workspace=ws)
+    torch.cuda.synchronize()
+    print(f"profile driver done: workload {workload}, M={M}, reps={reps}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,7 +475,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline only (no extra sections)")
+    ap.add_argument("--profile", nargs=3, type=int, metavar=("WORKLOAD", "M", "REPS"),
+                    help="profiling driver: one layer of WORKLOAD, every projection REPS times")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(*args.profile)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
