@@ -166,6 +166,40 @@ AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const 
                             int64_t N, uint16_t *Y, void *workspace, size_t workspace_bytes,
                             int32_t *dev_status, awq_stream_t stream);
 
+/*
+ * awq_w4a16_gemm_noalloc -- awq_w4a16_gemm for callers that cannot hand the
+ * library a workspace.  No counterpart in the AWQ paper or pages: this is an
+ * integration entry point of this library only.
+ *
+ * Who needs it: code that is not allowed to allocate device memory at the point
+ * where it runs the layer -- for example an inference-engine plugin whose
+ * execute callback may only use memory the engine planned beforehand, a
+ * real-time or fixed-budget deployment that allocates everything at start-up,
+ * or a plain C caller that has no device allocator of its own.  Instead of a
+ * caller-provided workspace, X / s is staged in a fixed scratch array that is
+ * part of the library's device image: AWQ_NOALLOC_SCRATCH_BYTES on every GPU
+ * that loads the library, held until the process exits.  The call itself
+ * allocates nothing (no cudaMalloc, no allocating library routine).
+ *
+ * Arguments, layouts, tolerance and errors are those of awq_w4a16_gemm, minus
+ * the workspace.  Limit: awq_w4a16_gemm_workspace_size(M, K, N) must not exceed
+ * AWQ_NOALLOC_SCRATCH_BYTES (2 * M * K bytes for M > 1, i.e. M * K <= 2 Mi
+ * elements); larger problems return AWQ_ERR_WORKSPACE before anything runs.
+ * Set-up: the first call on each device (with that device current) looks up
+ * the scratch array's device address; make that first call before any stream
+ * capture begins.
+ * Sharing: every call on a device uses the same scratch array, which keeps the
+ * last call's contents (nothing in it needs to start at zero: each call writes
+ * the part it reads).  Calls whose executions overlap on the GPU (different
+ * streams without ordering between them) race on the scratch array and give
+ * undefined results; order them on one stream or with events.
+ */
+#define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+AWQ_API awq_status_t awq_w4a16_gemm_noalloc(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                                            const uint16_t *scales, const int32_t *zeros,
+                                            int64_t M, int64_t K, int64_t N, uint16_t *Y,
+                                            int32_t *dev_status, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,8 +38,9 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_ARCH, ERR_CUDA, ERR_TIMEO
 SYMBOLS = (
     "awq_status_string", "awq_abi_version", "awq_act_stats", "awq_compute_scales",
     "awq_quantize_pack", "awq_w4a16_gemv_workspace_size", "awq_w4a16_gemv",
-    "awq_w4a16_gemm_workspace_size", "awq_w4a16_gemm",
+    "awq_w4a16_gemm_workspace_size", "awq_w4a16_gemm", "awq_w4a16_gemm_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class AwqError(RuntimeError):
@@ -74,8 +75,9 @@ def lib() -> ctypes.CDLL:
         L.awq_w4a16_gemm_workspace_size.argtypes = [I64, I64, I64]
         L.awq_w4a16_gemm_workspace_size.restype = SZ
         L.awq_w4a16_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, SZ, P, P]
+        L.awq_w4a16_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P]
         for name in ("awq_act_stats", "awq_compute_scales", "awq_quantize_pack",
-                     "awq_w4a16_gemv", "awq_w4a16_gemm"):
+                     "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_w4a16_gemm_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib

@@ -161,6 +161,31 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
 
 }  // namespace
 
+namespace awq {
+// The host-side argument checks of the matmul (null, shape, alignment), for
+// entry points that must reject bad arguments before any device query.
+awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                                const uint16_t *scales, const int32_t *zeros, int64_t M,
+                                int64_t K, int64_t N, const uint16_t *Y, const int32_t *dev_status)
+{
+    if (!X || !s || !Q || !scales || !zeros || !Y) return AWQ_ERR_NULL;
+    if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
+        !aligned16(Y) || (dev_status && !aligned4(dev_status)))
+        return AWQ_ERR_ALIGN;
+    return AWQ_OK;
+}
+
+// The workspace-taking matmul, for the library's other entry points.
+awq_status_t matmul_with_workspace(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                                   const uint16_t *scales, const int32_t *zeros, int64_t M,
+                                   int64_t K, int64_t N, uint16_t *Y, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, awq_stream_t stream)
+{
+    return run_matmul(X, s, Q, scales, zeros, M, K, N, Y, ws, ws_bytes, dev_status, stream);
+}
+}  // namespace awq
+
 extern "C" {
 
 const char *awq_status_string(awq_status_t status)

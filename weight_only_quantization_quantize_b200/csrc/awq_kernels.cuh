@@ -43,4 +43,15 @@ cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensor
                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                       int32_t *status, cudaStream_t st);
 
+// abi.cu -- host-side argument checks of the matmul (null, shape, alignment)
+awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                                const uint16_t *scales, const int32_t *zeros, int64_t M,
+                                int64_t K, int64_t N, const uint16_t *Y, const int32_t *dev_status);
+
+// abi.cu -- the matmul behind awq_w4a16_gemm, with an explicit workspace
+awq_status_t matmul_with_workspace(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                                   const uint16_t *scales, const int32_t *zeros, int64_t M,
+                                   int64_t K, int64_t N, uint16_t *Y, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, awq_stream_t stream);
+
 }  // namespace awq
