@@ -67,7 +67,8 @@ awq_status_t device_ready(int *sms)
                 }
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
-            if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess) {
+            if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
+                awq::configure_gemv() != cudaSuccess) {
                 cudaGetLastError();
                 return AWQ_ERR_CUDA;
             }
@@ -130,6 +131,13 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
     __half *Xp = reinterpret_cast<__half *>(ws);
 
     CUtensorMap tmQ, tmX;
+    awq::GemvPlan gplan;
+    if (M <= 8 && awq::plan_gemv(m, k, n, sms, &gplan)) {
+        if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return AWQ_ERR_CUDA;
+        return from_cuda(awq::launch_gemv(gplan, tmQ, hX, hs, hsc, zeros, hY, m, k, n, dev_status, st));
+    }
     if (M < 64) {
         const awq::SmallMPlan plan = awq::plan_small_m(m, k, n, sms);
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,

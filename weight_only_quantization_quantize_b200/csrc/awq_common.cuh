@@ -106,6 +106,33 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
         : "memory");
 }
 
+// Hint the hardware to pull a 2-D tile into L2 (no shared-memory destination,
+// no completion to wait for).  Safe before griddepcontrol.wait: L2 is the
+// coherence point, so data a predecessor writes later is still seen by the
+// real loads issued after the wait.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Allow the next kernel on the stream to start launching (its own prologue
+// then overlaps this kernel's tail).
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grids this kernel depends on have completed and their memory
+// is visible.  No global memory written by a predecessor may be read before.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 // src_bytes == 0 zero-fills the destination without reading global memory.
 __device__ __forceinline__ void cp_async_4(void *dst, const void *src, uint32_t src_bytes)
@@ -183,7 +210,7 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr)
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -197,15 +224,30 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // 1024 + z (or scaling by 1/16 and subtracting 64 + z) leaves q - z exactly.
 // Output pairs (low, high half): d[0] = (q0, q4), d[1] = (q1, q5),
 // d[2] = (q2, q6), d[3] = (q3, q7), each minus z.
+// The masks, the magic and 1/16 arrive as run-time values (UnpackConsts in
+// the kernel parameters): as literals the compiler re-materializes them before
+// every use, since a LOP3 encodes only one 32-bit immediate.
+struct UnpackConsts {
+    uint32_t mask_lo;    // 0x000F000F
+    uint32_t mask_hi;    // 0x00F000F0
+    uint32_t magic;      // 0x64006400 = (1024, 1024)
+    uint32_t sixteenth;  // 0x2C002C00 = (1/16, 1/16)
+};
+
+__host__ __device__ inline UnpackConsts unpack_consts()
+{
+    return UnpackConsts{0x000F000Fu, 0x00F000F0u, 0x64006400u, 0x2C002C00u};
+}
+
 __device__ __forceinline__ void unpack_minus_zero(uint32_t w, uint32_t za, uint32_t zb,
-                                                  uint32_t (&d)[4])
+                                                  uint32_t (&d)[4], const UnpackConsts &k)
 {
     const uint32_t w8 = w >> 8;
-    const uint32_t v0 = (w & 0x000F000Fu) | 0x64006400u;
-    const uint32_t v1 = (w & 0x00F000F0u) | 0x64006400u;
-    const uint32_t v2 = (w8 & 0x000F000Fu) | 0x64006400u;
-    const uint32_t v3 = (w8 & 0x00F000F0u) | 0x64006400u;
-    const uint32_t sixteenth = 0x2C002C00u;  // (1/16, 1/16)
+    const uint32_t v0 = (w & k.mask_lo) | k.magic;
+    const uint32_t v1 = (w & k.mask_hi) | k.magic;
+    const uint32_t v2 = (w8 & k.mask_lo) | k.magic;
+    const uint32_t v3 = (w8 & k.mask_hi) | k.magic;
+    const uint32_t sixteenth = k.sixteenth;
     asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d[0]) : "r"(v0), "r"(za));
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d[1]) : "r"(v1), "r"(sixteenth), "r"(zb));
     asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d[2]) : "r"(v2), "r"(za));

@@ -14,6 +14,22 @@ cudaError_t launch_quantize_pack(const __half *W, const __half *s, int K, int N,
                                  __half *scales, int32_t *zeros, int32_t *status,
                                  cudaStream_t st);
 
+// gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group
+struct GemvPlan {
+    int splits;       // CTAs per cluster along K
+    int n_tiles;      // 128-column tiles
+    int kh;           // consumer warps per 32-column slab
+    int stages;
+    int xpro_bytes;
+    int gmeta_bytes;
+    size_t smem;
+};
+bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *plan);
+cudaError_t configure_gemv();
+cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __half *X,
+                        const __half *s, const __half *scales, const int32_t *zeros, __half *Y,
+                        int M, int K, int N, int32_t *status, cudaStream_t st);
+
 // matmul_small.cu -- M < 64: register-fed tensor cores, TMA weight stream
 struct SmallMPlan {
     int mt;          // token tiles of 8
@@ -21,6 +37,7 @@ struct SmallMPlan {
     int splits;      // CTAs per cluster along K
     int n_tiles;     // 128-column tiles
     int stages;
+    int kh;          // consumer warps per 32-column slab (k split inside a group)
     size_t smem;     // dynamic shared memory bytes
 };
 SmallMPlan plan_small_m(int M, int K, int N, int num_sms);

@@ -1,0 +1,446 @@
+// gemv.cu -- Y = (X / s) . dequant(Q) for M <= 8 tokens: the single-token
+// decode GEMV (and the smallest batches), the HBM-bound regime.
+//
+// Sources: lansai AWQ explainer (ai.lansai.wang/107648), "AWQ 的四步链路"
+// (Y = (X/s)(sW)); "Awq Quantization" (skillselion.com), "WQLinear Kernel
+// Variants" (a GEMV kernel for batch size 1), "Group Size Configuration" and
+// "Zero-Point Quantization" (4-bit codes, groups of 128, zero point).
+//
+// Every packed weight is read once from HBM.  To keep the per-weight work at a
+// handful of integer ops, the zero point and the step leave the inner loop:
+// with S0 / S1 the sums of X' over the group's even / odd k (k mod 8), and
+// R0 = sum_{k even} x'_k (1024 + q_k),  R1 = sum_{k odd} x'_k (1024 + 16 q_k)
+// (what the tensor cores produce when fed the raw OR-ed nibbles),
+//   sum_k x'_k (q_k - z) = R0 + R1 / 16 - (1024 S0 + 64 S1) - z (S0 + S1),
+// and the group's step multiplies that once.  S0, S1 are computed per CTA in
+// the prologue together with X' = fp16(X / s), from the same rounded values.
+//
+// Structure (one CTA = 128 output columns x a k range; clusters split K):
+//   producer warp   TMA ring of 128-row groups (four 16 x 32-word boxes,
+//                   128-byte swizzle) + cp.async of the group's steps and zero
+//                   words; before the dependency wait it warms L2 with the
+//                   CTA's packed weights (programmatic dependent launch).
+//   4*KH consumers  32 columns per warp (KH warps split a group's rows); a
+//                   lane turns one 16-byte load (4 columns x 8 k) into four
+//                   even-form and four odd-form f16x2 operands with LOP3 only
+//                   and feeds mma.sync m16n8k16 in swap-AB form (columns are
+//                   MMA rows, tokens MMA columns).
+//   epilogue        per-warp partials -> shared memory -> reduced across the
+//                   cluster through distributed shared memory in rank order.
+#include "awq_kernels.cuh"
+
+namespace awq {
+
+namespace {
+
+constexpr int kBN = 128;
+constexpr int kQStage = 4 * 2048;
+constexpr int kStageBytes = 9216;  // 8 KB words + 256 B steps + 64 B zero words, padded
+constexpr int kRedPitch = 132;
+constexpr int kSmemOptIn = 232448;
+
+struct GemvParams {
+    const __half *X;
+    const __half *s;
+    const __half *scales;
+    const int32_t *zeros;
+    __half *Y;
+    int32_t *status;
+    int M, K, N, G, splits;
+    int xpro_bytes;   // X' buffer: M * chunks * 16
+    int gmeta_bytes;  // per (token, group, half): {1024 S0 + 64 S1, S0 + S1}
+    // Unpack constants, passed at run time: as compile-time literals the
+    // compiler re-materializes them before every use (a LOP3 encodes only one
+    // 32-bit immediate), which nearly doubles the integer-pipe work per weight.
+    uint32_t mask_lo;  // 0x000F000F: nibbles 0 and 4 (after >> 8: 2 and 6)
+    uint32_t mask_hi;  // 0x00F000F0: nibbles 1 and 5 (after >> 8: 3 and 7)
+    uint32_t magic;    // 0x64006400: binary16 1024.0 in both halves
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+template <int S, int KH>
+__global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmQ, const GemvParams p)
+{
+    constexpr int kConsumers = 4 * KH;
+    constexpr int kCThreads = 32 * kConsumers;
+    constexpr int kAllThreads = kCThreads + 32;
+    constexpr int kSteps = 4 / KH;
+
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *smem = align1024(smem_dyn);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int split = blockIdx.x;
+    const int n0 = blockIdx.y * kBN;
+    const int g_begin = static_cast<int>(static_cast<int64_t>(split) * p.G / p.splits);
+    const int g_end = static_cast<int>(static_cast<int64_t>(split + 1) * p.G / p.splits);
+    const int ng = g_end - g_begin;
+    const int chunks = ng * 16;
+
+    pdl_launch_dependents();
+
+    uint8_t *xpro = smem + S * kStageBytes;
+    float2 *gmeta = reinterpret_cast<float2 *>(xpro + p.xpro_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.xpro_bytes + p.gmeta_bytes);
+    uint64_t *empty = full + S;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1 + 32);
+            mbar_init(&empty[i], kConsumers);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    float acc[2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[a][i] = 0.0f;
+
+    if (warp == kConsumers) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            const int npf = ng < 64 ? ng : 64;
+            for (int it = 0; it < npf; ++it)
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    tma_prefetch_l2_2d(&tmQ, n0 + 32 * w, (g_begin + it) * 16);
+        }
+        pdl_wait();
+        bool ok = true;
+        for (int it = 0; it < ng; ++it) {
+            const int st = it % S;
+            if (it >= S && !mbar_wait(&empty[st], ((it / S) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t *stg = smem + st * kStageBytes;
+            const int g = g_begin + it;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[st], kQStage);
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    tma_load_2d(stg + w * 2048, &tmQ, &full[st], n0 + 32 * w, g * 16);
+            }
+            uint8_t *meta = stg + kQStage;
+            if (lane < 16) {
+                const int n = n0 + 8 * lane;
+                const bool in = n < p.N;
+                cp_async_16(meta + 16 * lane, p.scales + static_cast<size_t>(g) * p.N + (in ? n : 0),
+                            in ? 16u : 0u);
+            } else {
+                const int wi = n0 / 8 + (lane - 16);
+                const bool in = wi < p.N / 8;
+                cp_async_4(meta + 256 + 4 * (lane - 16),
+                           p.zeros + static_cast<size_t>(g) * (p.N / 8) + (in ? wi : 0), in ? 4u : 0u);
+            }
+            cp_async_arrive_noinc(&full[st]);
+        }
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    } else {
+        // ------------------------------------------------------------ consumers
+        pdl_wait();
+        // Prologue: X' = fp16(X / s) for this CTA's k range, stored per 8-channel
+        // chunk in the order (0,4),(2,6),(1,5),(3,7) (even-form pairs, then
+        // odd-form pairs), plus the per-(token, group, half) sums of X'.
+        {
+            constexpr int kLanesPerHalf = 16 / KH;  // chunks per group half
+            const int sub = lane >> 4;              // two (token, group) pairs per warp pass
+            const int c16 = lane & 15;
+            const int pairs = p.M * ng;
+            for (int base = warp * 2; base < pairs; base += 2 * kConsumers) {
+                const int pair = base + sub;
+                const bool valid = pair < pairs;
+                const int tok = valid ? pair / ng : 0;
+                const int gl = valid ? pair - tok * ng : 0;
+                float e = 0.0f, o = 0.0f;
+                if (valid) {
+                    const int ch = gl * 16 + c16;
+                    const int k = (g_begin + gl) * kGroup + c16 * 8;
+                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(tok) * p.K + k));
+                    const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(p.s + k));
+                    const __half *xh = reinterpret_cast<const __half *>(&xv);
+                    const __half *sh = reinterpret_cast<const __half *>(&sv);
+                    __half q[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        q[j] = __float2half_rn(__fdiv_rn(__half2float(xh[j]), __half2float(sh[j])));
+                    e = (__half2float(q[0]) + __half2float(q[2])) + (__half2float(q[4]) + __half2float(q[6]));
+                    o = (__half2float(q[1]) + __half2float(q[3])) + (__half2float(q[5]) + __half2float(q[7]));
+                    uint4 r;
+                    r.x = __half_as_ushort(q[0]) | (static_cast<uint32_t>(__half_as_ushort(q[4])) << 16);
+                    r.y = __half_as_ushort(q[2]) | (static_cast<uint32_t>(__half_as_ushort(q[6])) << 16);
+                    r.z = __half_as_ushort(q[1]) | (static_cast<uint32_t>(__half_as_ushort(q[5])) << 16);
+                    r.w = __half_as_ushort(q[3]) | (static_cast<uint32_t>(__half_as_ushort(q[7])) << 16);
+                    *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok) * chunks + (ch ^ (tok & 7))) * 16) = r;
+                }
+                // butterfly over the lanes of one group half (fixed order)
+#pragma unroll
+                for (int off = kLanesPerHalf / 2; off > 0; off >>= 1) {
+                    e += __shfl_xor_sync(0xffffffffu, e, off);
+                    o += __shfl_xor_sync(0xffffffffu, o, off);
+                }
+                if (valid && (c16 % kLanesPerHalf) == 0)
+                    gmeta[(tok * ng + gl) * KH + c16 / kLanesPerHalf] =
+                        make_float2(fmaf(1024.0f, e, 64.0f * o), e + o);
+            }
+            named_bar_sync(1, kCThreads);
+        }
+
+        const int gq = lane >> 2;
+        const int t = lane & 3;
+        const int slab = warp & 3;
+        const int khalf = warp >> 2;
+        const int colw = 32 * slab + 4 * gq;
+        const int tok0 = 2 * t;
+        const uint8_t *xbase = xpro;
+        const uint32_t mlo = p.mask_lo, mhi = p.mask_hi, magic = p.magic;
+        bool ok = true;
+        for (int it = 0; it < ng; ++it) {
+            const int st = it % S;
+            if (!mbar_wait(&full[st], (it / S) & 1)) {
+                ok = false;
+                break;
+            }
+            const uint8_t *stg = smem + st * kStageBytes;
+            const uint8_t *meta = stg + kQStage;
+            const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
+            const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
+
+            float R[2][2][4];  // [tile][form][c]
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int f = 0; f < 2; ++f)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) R[a][f][i] = 0.0f;
+
+            const uint8_t *qslab = stg + slab * 2048;
+#pragma unroll
+            for (int ss = 0; ss < kSteps; ++ss) {
+                const int sidx = khalf * kSteps + ss;
+                const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);
+                const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
+                uint4 bx = make_uint4(0u, 0u, 0u, 0u);
+                if (gq < p.M)
+                    bx = *reinterpret_cast<const uint4 *>(
+                        xbase + (static_cast<size_t>(gq) * chunks + ((it * 16 + r) ^ gq)) * 16);
+                const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+                uint32_t ev0[4], ev2[4], od1[4], od3[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t w8 = w[c] >> 8;
+                    ev0[c] = (w[c] & mlo) | magic;  // 1024 + q0, 1024 + q4
+                    ev2[c] = (w8 & mlo) | magic;    // 1024 + q2, 1024 + q6
+                    od1[c] = (w[c] & mhi) | magic;  // 1024 + 16 q1, 1024 + 16 q5
+                    od3[c] = (w8 & mhi) | magic;    // 1024 + 16 q3, 1024 + 16 q7
+                }
+#pragma unroll
+                for (int tile = 0; tile < 2; ++tile) {
+                    const int c0 = 2 * tile, c1 = 2 * tile + 1;
+                    const uint32_t ae[4] = {ev0[c0], ev0[c1], ev2[c0], ev2[c1]};
+                    const uint32_t ao[4] = {od1[c0], od1[c1], od3[c0], od3[c1]};
+                    mma_16816(R[tile][0], ae, bx.x, bx.y);
+                    mma_16816(R[tile][1], ao, bx.z, bx.w);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+
+            // group epilogue: y += step * (R0 + R1/16 - (1024 S0 + 64 S1) - z (S0 + S1))
+            const float2 gm0 = tok0 < p.M ? gmeta[(tok0 * ng + it) * KH + khalf] : make_float2(0.f, 0.f);
+            const float2 gm1 = tok0 + 1 < p.M ? gmeta[((tok0 + 1) * ng + it) * KH + khalf] : make_float2(0.f, 0.f);
+            const int zsh = (colw & 7) * 4;
+            const __half2 s01 = *reinterpret_cast<const __half2 *>(&sc.x);
+            const __half2 s23 = *reinterpret_cast<const __half2 *>(&sc.y);
+            const float stp[4] = {__low2float(s01), __high2float(s01), __low2float(s23), __high2float(s23)};
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = 2 * tile + (i >> 1);
+                    const float z = static_cast<float>((zw >> (zsh + 4 * c)) & 15u);
+                    const float2 gm = (i & 1) ? gm1 : gm0;
+                    float pgrp = fmaf(R[tile][1][i], 0.0625f, R[tile][0][i]) - gm.x;
+                    pgrp = fmaf(-z, gm.y, pgrp);
+                    acc[tile][i] = fmaf(stp[c], pgrp, acc[tile][i]);
+                }
+        }
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    __syncthreads();
+    float *red = reinterpret_cast<float *>(smem);  // [khalf][token 0..7][column]
+    constexpr int kHalfStride = 8 * kRedPitch;
+    if (warp < kConsumers) {
+        const int gq = lane >> 2, t = lane & 3;
+        const int colw = 32 * (warp & 3) + 4 * gq;
+        float *rh = red + (warp >> 2) * kHalfStride;
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const int tok = 2 * t;
+            const int col = colw + 2 * tile;
+            rh[tok * kRedPitch + col] = acc[tile][0];
+            rh[(tok + 1) * kRedPitch + col] = acc[tile][1];
+            rh[tok * kRedPitch + col + 1] = acc[tile][2];
+            rh[(tok + 1) * kRedPitch + col + 1] = acc[tile][3];
+        }
+    }
+    cluster_sync_all();
+    const uint32_t red_base = smem_u32(red);
+    for (int e = threadIdx.x; e < p.M * 16; e += kAllThreads) {
+        const int tok = e >> 4;
+        const int ch = e & 15;
+        const int n = n0 + ch * 8;
+        if (ch % p.splits != split || n >= p.N) continue;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        for (int r = 0; r < p.splits; ++r) {
+#pragma unroll
+            for (int h = 0; h < KH; ++h) {
+                const uint32_t off = red_base + (h * kHalfStride + tok * kRedPitch + ch * 8) * 4;
+                const uint32_t a = map_to_rank(off, r);
+                const float4 lo = ld_cluster_f4(a);
+                const float4 hi = ld_cluster_f4(a + 16);
+                v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+                v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
+            }
+        }
+        uint4 o;
+        o.x = __half_as_ushort(__float2half_rn(v[0])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
+        o.y = __half_as_ushort(__float2half_rn(v[2])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[3]))) << 16);
+        o.z = __half_as_ushort(__float2half_rn(v[4])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[5]))) << 16);
+        o.w = __half_as_ushort(__float2half_rn(v[6])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[7]))) << 16);
+        *reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(tok) * p.N + n) = o;
+    }
+    cluster_sync_all();
+}
+
+template <int S, int KH>
+cudaError_t launch_gemv_one(const GemvPlan &plan, const CUtensorMap &tmQ, const GemvParams &prm,
+                            cudaStream_t st)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.splits, plan.n_tiles, 1);
+    cfg.blockDim = dim3(32 * (4 * KH + 1), 1, 1);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = plan.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<S, KH>, tmQ, prm);
+}
+
+template <int S, int KH>
+cudaError_t configure_gemv_one()
+{
+    return cudaFuncSetAttribute(gemv_kernel<S, KH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemOptIn);
+}
+
+}  // namespace
+
+cudaError_t configure_gemv()
+{
+    const cudaError_t r[] = {configure_gemv_one<8, 1>(), configure_gemv_one<8, 2>(),
+                             configure_gemv_one<4, 1>(), configure_gemv_one<4, 2>()};
+    for (cudaError_t x : r)
+        if (x != cudaSuccess) return x;
+    return cudaSuccess;
+}
+
+#ifdef AWQ_TUNING
+static int tune_env(const char *name, int dflt)
+{
+    const char *v = getenv(name);
+    return v ? atoi(v) : dflt;
+}
+#endif
+
+bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
+{
+    if (M < 1 || M > 8) return false;
+    const int G = K / kGroup;
+    const int max_split = G < 8 ? G : 8;
+    pl->n_tiles = (N + kBN - 1) / kBN;
+    pl->kh = 1;
+    // Measured on the decode shapes: split K until there are about six CTAs
+    // per SM (splits dividing the group count); with four or more CTAs per SM
+    // a 4-deep ring keeps enough bytes in flight, below that 8 stages do.
+    int splits = max_split;
+    for (int sp = 1; sp <= max_split; ++sp) {
+        if (pl->n_tiles * sp >= 6 * num_sms && (G % sp == 0)) {
+            splits = sp;
+            break;
+        }
+    }
+    pl->stages = pl->n_tiles * splits >= 4 * num_sms ? 4 : 8;
+#ifdef AWQ_TUNING
+    splits = tune_env("AWQ_TUNE_SPLITS", splits);
+    if (splits > max_split) splits = max_split;
+    if (splits < 1) splits = 1;
+    pl->kh = tune_env("AWQ_TUNE_KH", pl->kh);
+    pl->stages = tune_env("AWQ_TUNE_STAGES", pl->stages) <= 4 ? 4 : 8;
+#endif
+    // X' and the group sums live in shared memory: M * (groups per CTA) * 256 B
+    // (+ 8 B per group half); find the smallest split at or above the choice that fits
+    for (; splits <= max_split; ++splits) {
+        const int gmax = (G + splits - 1) / splits;
+        if (static_cast<size_t>(M) * gmax * (256 + 8 * pl->kh) <= 64 * 1024) break;
+    }
+    if (splits > max_split) return false;
+    pl->splits = splits;
+    const int gmax = (G + splits - 1) / splits;
+    pl->xpro_bytes = M * gmax * 256;
+    pl->gmeta_bytes = (M * gmax * pl->kh * 8 + 15) & ~15;
+    pl->smem = 1024 + static_cast<size_t>(pl->stages) * kStageBytes + pl->xpro_bytes + pl->gmeta_bytes +
+               2 * pl->stages * sizeof(uint64_t);
+    return true;
+}
+
+cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __half *X,
+                        const __half *s, const __half *scales, const int32_t *zeros, __half *Y,
+                        int M, int K, int N, int32_t *status, cudaStream_t st)
+{
+    GemvParams prm{};
+    prm.X = X;
+    prm.s = s;
+    prm.scales = scales;
+    prm.zeros = zeros;
+    prm.Y = Y;
+    prm.status = status;
+    prm.M = M;
+    prm.K = K;
+    prm.N = N;
+    prm.G = K / kGroup;
+    prm.splits = plan.splits;
+    prm.xpro_bytes = plan.xpro_bytes;
+    prm.gmeta_bytes = plan.gmeta_bytes;
+    prm.mask_lo = 0x000F000Fu;
+    prm.mask_hi = 0x00F000F0u;
+    prm.magic = 0x64006400u;
+    if (plan.stages == 4)
+        return plan.kh == 2 ? launch_gemv_one<4, 2>(plan, tmQ, prm, st)
+                            : launch_gemv_one<4, 1>(plan, tmQ, prm, st);
+    return plan.kh == 2 ? launch_gemv_one<8, 2>(plan, tmQ, prm, st)
+                        : launch_gemv_one<8, 1>(plan, tmQ, prm, st);
+}
+
+}  // namespace awq

@@ -35,7 +35,6 @@ namespace awq {
 
 namespace {
 
-constexpr int kThreads = 160;       // 4 consumer warps + 1 producer warp
 constexpr int kBN = 128;            // output columns per CTA
 constexpr int kQStage = 4 * 2048;   // 4 boxes of [16 rows x 32 words]
 constexpr int kMetaBytes = 256 + 64;  // 128 scales + 16 zero words
@@ -56,6 +55,7 @@ struct Params {
     int xbox;          // bytes reserved per staged X' box (0 with the prologue)
     int stage_bytes;
     int prologue_bytes;
+    UnpackConsts uk;
 };
 
 // x / s for 8 consecutive channels, rounded to binary16, stored in the
@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(256) prescale_kernel(const __half *__restrict_
                                                       const __half *__restrict__ s, int64_t chunks,
                                                       int kchunks, __half *__restrict__ Xp)
 {
+    pdl_launch_dependents();
+    pdl_wait();  // X may come from the previous kernel on the stream
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= chunks) return;
     const int kc = static_cast<int>(i % kchunks);
@@ -93,11 +95,19 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <int MT, bool PRO, int S>
-__global__ void __launch_bounds__(kThreads, 1)
+// KH = warps per 32-column slab: with KH = 2 a warp pair splits each group's
+// 128 rows (k 0..63 and 64..127), doubling the warps that hide MMA and
+// shared-memory latency; the halves are summed in the epilogue.
+template <int MT, bool PRO, int S, int KH>
+__global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     small_m_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmX,
                    const Params p)
 {
+    constexpr int kConsumers = 4 * KH;
+    constexpr int kCThreads = 32 * kConsumers;
+    constexpr int kAllThreads = kCThreads + 32;
+    constexpr int kSteps = 4 / KH;  // 32-row steps per warp per group
+
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *smem = align1024(smem_dyn);
     const int warp = threadIdx.x >> 5;
@@ -109,14 +119,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ng = g_end - g_begin;
     const int chunks = ng * 16;  // 8-channel chunks of this CTA's k range
 
+    // the next kernel on the stream may begin its own prologue now
+    pdl_launch_dependents();
+
     uint8_t *xpro = smem + S * p.stage_bytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.prologue_bytes);
     uint64_t *empty = full + S;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1 + 32);  // expect_tx arrival + 32 cp.async arrivals
-            mbar_init(&empty[i], 4);      // one per consumer warp
+            mbar_init(&full[i], 1 + 32);     // expect_tx arrival + 32 cp.async arrivals
+            mbar_init(&empty[i], kConsumers);  // one per consumer warp
         }
         fence_barrier_init();
     }
@@ -130,12 +143,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[a][j][i] = 0.0f;
 
-    if (warp == 4) {
+    if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             if (!PRO) prefetch_tmap(&tmX);
+            // Warm L2 with this CTA's packed weights while the previous kernel
+            // on the stream finishes; the real loads below come after the wait.
+            const int npf = ng < 64 ? ng : 64;
+            for (int it = 0; it < npf; ++it)
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    tma_prefetch_l2_2d(&tmQ, n0 + 32 * w, (g_begin + it) * 16);
         }
+        pdl_wait();
         const uint32_t tx = kQStage + (PRO ? 0 : 2 * p.M * 128);
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
@@ -175,10 +196,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ consumers
         const int gq = lane >> 2;
         const int t = lane & 3;
-        const int colw = 32 * warp + 4 * gq;  // my 4 columns: colw .. colw+3 (tile-local)
+        const int slab = warp & 3;
+        const int khalf = warp >> 2;            // 0 when KH == 1
+        const int colw = 32 * slab + 4 * gq;    // my 4 columns: colw .. colw+3 (tile-local)
+        pdl_wait();
         if (PRO) {
             const int total = p.M * chunks;
-            for (int idx = threadIdx.x; idx < total; idx += 128) {
+            for (int idx = threadIdx.x; idx < total; idx += kCThreads) {
                 const int tok = idx / chunks;
                 const int ch = idx - tok * chunks;
                 const int k = g_begin * kGroup + ch * 8;
@@ -187,9 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok) * chunks + (ch ^ (tok & 7))) * 16) =
                     prescale8(xv, sv);
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kCThreads);
         }
         const uint32_t xpro_base = smem_u32(xpro);
+        const UnpackConsts uk = p.uk;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
             const int st = it % S;
@@ -206,18 +231,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) zero_constants((zw >> (zsh + 4 * c)) & 15u, za[c], zb[c]);
 
-            float grp[2][MT][4];
+            // with few token tiles, two accumulator sets (even / odd step) halve the
+            // MMA dependency chains; more token tiles already give independent chains
+            constexpr int kSets = MT <= 2 ? 2 : 1;
+            float grp[kSets][2][MT][4];
 #pragma unroll
-            for (int a = 0; a < 2; ++a)
+            for (int b = 0; b < kSets; ++b)
 #pragma unroll
-                for (int j = 0; j < MT; ++j)
+                for (int a = 0; a < 2; ++a)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) grp[a][j][i] = 0.0f;
+                    for (int j = 0; j < MT; ++j)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) grp[b][a][j][i] = 0.0f;
 
-            const uint32_t qslab = smem_u32(stg) + warp * 2048;
+            const uint32_t qslab = smem_u32(stg) + slab * 2048;
             const uint32_t xstage = smem_u32(stg) + kQStage;
 #pragma unroll
-            for (int sidx = 0; sidx < 4; ++sidx) {
+            for (int ss = 0; ss < kSteps; ++ss) {
+                const int sidx = khalf * kSteps + ss;
                 const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);  // packed row in the group
                 const uint4 wq = lds128(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
                 uint32_t bx[MT][4];
@@ -240,10 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 uint32_t d[4][4];
-                unpack_minus_zero(wq.x, za[0], zb[0], d[0]);
-                unpack_minus_zero(wq.y, za[1], zb[1], d[1]);
-                unpack_minus_zero(wq.z, za[2], zb[2], d[2]);
-                unpack_minus_zero(wq.w, za[3], zb[3], d[3]);
+                unpack_minus_zero(wq.x, za[0], zb[0], d[0], uk);
+                unpack_minus_zero(wq.y, za[1], zb[1], d[1], uk);
+                unpack_minus_zero(wq.z, za[2], zb[2], d[2], uk);
+                unpack_minus_zero(wq.w, za[3], zb[3], d[3], uk);
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
                     const uint32_t a0[4] = {d[2 * tile][0], d[2 * tile + 1][0], d[2 * tile][1],
@@ -252,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             d[2 * tile + 1][3]};
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
-                        mma_16816(grp[tile][j], a0, bx[j][0], bx[j][1]);
-                        mma_16816(grp[tile][j], a1, bx[j][2], bx[j][3]);
+                        mma_16816(grp[ss % kSets][tile][j], a0, bx[j][0], bx[j][1]);
+                        mma_16816(grp[ss % kSets][tile][j], a1, bx[j][2], bx[j][3]);
                     }
                 }
             }
@@ -263,42 +294,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sc.y));
 #pragma unroll
             for (int j = 0; j < MT; ++j) {
-                acc[0][j][0] = fmaf(s01.x, grp[0][j][0], acc[0][j][0]);
-                acc[0][j][1] = fmaf(s01.x, grp[0][j][1], acc[0][j][1]);
-                acc[0][j][2] = fmaf(s01.y, grp[0][j][2], acc[0][j][2]);
-                acc[0][j][3] = fmaf(s01.y, grp[0][j][3], acc[0][j][3]);
-                acc[1][j][0] = fmaf(s23.x, grp[1][j][0], acc[1][j][0]);
-                acc[1][j][1] = fmaf(s23.x, grp[1][j][1], acc[1][j][1]);
-                acc[1][j][2] = fmaf(s23.y, grp[1][j][2], acc[1][j][2]);
-                acc[1][j][3] = fmaf(s23.y, grp[1][j][3], acc[1][j][3]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float f0 = i < 2 ? s01.x : s01.y;
+                    const float f1 = i < 2 ? s23.x : s23.y;
+                    float p0 = grp[0][0][j][i], p1 = grp[0][1][j][i];
+                    if (kSets == 2) {
+                        p0 += grp[kSets - 1][0][j][i];
+                        p1 += grp[kSets - 1][1][j][i];
+                    }
+                    acc[0][j][i] = fmaf(f0, p0, acc[0][j][i]);
+                    acc[1][j][i] = fmaf(f1, p1, acc[1][j][i]);
+                }
             }
         }
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     }
 
     // ---------------------------------------------------------------- epilogue
-    __syncthreads();  // every stage consumed: the ring can hold the partial tile
+    __syncthreads();  // every stage consumed: the ring can hold the partial tiles
+    // red[khalf][token][column]
     float *red = reinterpret_cast<float *>(smem);
-    if (warp < 4) {
+    constexpr int kHalfStride = 8 * MT * kRedPitch;
+    if (warp < kConsumers) {
         const int gq = lane >> 2, t = lane & 3;
-        const int colw = 32 * warp + 4 * gq;
+        const int colw = 32 * (warp & 3) + 4 * gq;
+        float *rh = red + (warp >> 2) * kHalfStride;
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
             for (int j = 0; j < MT; ++j) {
                 const int tok = 8 * j + 2 * t;
                 const int col = colw + 2 * tile;
-                red[tok * kRedPitch + col] = acc[tile][j][0];
-                red[(tok + 1) * kRedPitch + col] = acc[tile][j][1];
-                red[tok * kRedPitch + col + 1] = acc[tile][j][2];
-                red[(tok + 1) * kRedPitch + col + 1] = acc[tile][j][3];
+                rh[tok * kRedPitch + col] = acc[tile][j][0];
+                rh[(tok + 1) * kRedPitch + col] = acc[tile][j][1];
+                rh[tok * kRedPitch + col + 1] = acc[tile][j][2];
+                rh[(tok + 1) * kRedPitch + col + 1] = acc[tile][j][3];
             }
     }
     cluster_sync_all();
     // this rank finishes the 8-column chunks ch with ch % splits == rank,
-    // summing the ranks' partials in rank order
+    // summing the partials in (rank, k-half) order
     const uint32_t red_base = smem_u32(red);
-    for (int e = threadIdx.x; e < p.M * 16; e += kThreads) {
+    for (int e = threadIdx.x; e < p.M * 16; e += kAllThreads) {
         const int tok = e >> 4;
         const int ch = e & 15;
         const int n = n0 + ch * 8;
@@ -306,13 +344,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-        const uint32_t off = red_base + (tok * kRedPitch + ch * 8) * 4;
         for (int r = 0; r < p.splits; ++r) {
-            const uint32_t a = map_to_rank(off, r);
-            const float4 lo = ld_cluster_f4(a);
-            const float4 hi = ld_cluster_f4(a + 16);
-            v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
-            v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
+#pragma unroll
+            for (int h = 0; h < KH; ++h) {
+                const uint32_t off = red_base + (h * kHalfStride + tok * kRedPitch + ch * 8) * 4;
+                const uint32_t a = map_to_rank(off, r);
+                const float4 lo = ld_cluster_f4(a);
+                const float4 hi = ld_cluster_f4(a + 16);
+                v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+                v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
+            }
         }
         uint4 o;
         o.x = __half_as_ushort(__float2half_rn(v[0])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
@@ -324,30 +365,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_sync_all();  // keep this CTA's partials alive until every rank has read them
 }
 
-template <int MT, bool PRO, int S>
+template <int MT, bool PRO, int S, int KH>
 cudaError_t launch_one(const SmallMPlan &plan, const CUtensorMap &tmQ, const CUtensorMap &tmX,
                        const Params &prm, cudaStream_t st)
 {
-    auto kern = small_m_kernel<MT, PRO, S>;
+    auto kern = small_m_kernel<MT, PRO, S, KH>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.splits, plan.n_tiles, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(32 * (4 * KH + 1), 1, 1);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = plan.splits;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tmQ, tmX, prm);
 }
 
-template <int MT, bool PRO, int S>
+template <int MT, bool PRO, int S, int KH>
 cudaError_t configure_one()
 {
-    return cudaFuncSetAttribute(small_m_kernel<MT, PRO, S>,
+    return cudaFuncSetAttribute(small_m_kernel<MT, PRO, S, KH>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemOptIn);
 }
 
@@ -357,15 +400,23 @@ cudaError_t configure_small_m()
 {
     cudaError_t e = cudaSuccess;
     const cudaError_t r[] = {
-        configure_one<1, true, stages_for(1)>(),  configure_one<1, false, stages_for(1)>(),
-        configure_one<2, false, stages_for(2)>(), configure_one<3, false, stages_for(3)>(),
-        configure_one<4, false, stages_for(4)>(), configure_one<5, false, stages_for(5)>(),
-        configure_one<6, false, stages_for(6)>(), configure_one<7, false, stages_for(7)>(),
-        configure_one<8, false, stages_for(8)>()};
+        configure_one<1, true, stages_for(1), 2>(),  configure_one<1, true, stages_for(1), 1>(),
+        configure_one<1, false, stages_for(1), 2>(), configure_one<2, false, stages_for(2), 2>(),
+        configure_one<3, false, stages_for(3), 2>(), configure_one<4, false, stages_for(4), 2>(),
+        configure_one<5, false, stages_for(5), 2>(), configure_one<6, false, stages_for(6), 2>(),
+        configure_one<7, false, stages_for(7), 2>(), configure_one<8, false, stages_for(8), 2>()};
     for (cudaError_t x : r)
         if (x != cudaSuccess) e = x;
     return e;
 }
+
+#ifdef AWQ_TUNING
+static int tune_env(const char *name, int dflt)
+{
+    const char *v = getenv(name);
+    return v ? atoi(v) : dflt;
+}
+#endif
 
 SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
 {
@@ -373,6 +424,7 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
     pl.mt = (M + 7) / 8;
     pl.n_tiles = (N + kBN - 1) / kBN;
     pl.stages = stages_for(pl.mt);
+    pl.kh = 2;
     const int G = K / kGroup;
     const int max_split = G < 8 ? G : 8;
     const int target = 2 * num_sms;
@@ -383,6 +435,12 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
             break;
         }
     }
+#ifdef AWQ_TUNING
+    splits = tune_env("AWQ_TUNE_SPLITS", splits);
+    if (splits > max_split) splits = max_split;
+    if (splits < 1) splits = 1;
+    if (pl.mt == 1) pl.kh = tune_env("AWQ_TUNE_KH", pl.kh);
+#endif
     pl.prologue = false;
     if (pl.mt == 1) {
         // X / s in shared memory needs M * (groups per split) * 256 bytes
@@ -395,6 +453,7 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
             }
         }
     }
+    if (!pl.prologue) pl.kh = 2;
     pl.splits = splits;
     const int xbox = pl.prologue ? 0 : ((M * 128 + 1023) & ~1023);
     const int stage_bytes = (kQStage + 2 * xbox + kMetaBytes + 1023) & ~1023;
@@ -410,8 +469,16 @@ cudaError_t launch_prescale(const __half *X, const __half *s, int M, int K, __ha
 {
     const int64_t chunks = static_cast<int64_t>(M) * (K / 8);
     const int64_t blocks = (chunks + 255) / 256;
-    prescale_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(X, s, chunks, K / 8, Xp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prescale_kernel, X, s, chunks, K / 8, Xp);
 }
 
 cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const CUtensorMap &tmX,
@@ -435,17 +502,20 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
     prm.stage_bytes = (kQStage + 2 * prm.xbox + kMetaBytes + 1023) & ~1023;
     const int gmax = (prm.G + plan.splits - 1) / plan.splits;
     prm.prologue_bytes = plan.prologue ? M * gmax * 256 : 0;
+    prm.uk = unpack_consts();
     switch (plan.mt) {
     case 1:
-        return plan.prologue ? launch_one<1, true, stages_for(1)>(plan, tmQ, tmX, prm, st)
-                             : launch_one<1, false, stages_for(1)>(plan, tmQ, tmX, prm, st);
-    case 2: return launch_one<2, false, stages_for(2)>(plan, tmQ, tmX, prm, st);
-    case 3: return launch_one<3, false, stages_for(3)>(plan, tmQ, tmX, prm, st);
-    case 4: return launch_one<4, false, stages_for(4)>(plan, tmQ, tmX, prm, st);
-    case 5: return launch_one<5, false, stages_for(5)>(plan, tmQ, tmX, prm, st);
-    case 6: return launch_one<6, false, stages_for(6)>(plan, tmQ, tmX, prm, st);
-    case 7: return launch_one<7, false, stages_for(7)>(plan, tmQ, tmX, prm, st);
-    case 8: return launch_one<8, false, stages_for(8)>(plan, tmQ, tmX, prm, st);
+        if (plan.prologue)
+            return plan.kh == 1 ? launch_one<1, true, stages_for(1), 1>(plan, tmQ, tmX, prm, st)
+                                : launch_one<1, true, stages_for(1), 2>(plan, tmQ, tmX, prm, st);
+        return launch_one<1, false, stages_for(1), 2>(plan, tmQ, tmX, prm, st);
+    case 2: return launch_one<2, false, stages_for(2), 2>(plan, tmQ, tmX, prm, st);
+    case 3: return launch_one<3, false, stages_for(3), 2>(plan, tmQ, tmX, prm, st);
+    case 4: return launch_one<4, false, stages_for(4), 2>(plan, tmQ, tmX, prm, st);
+    case 5: return launch_one<5, false, stages_for(5), 2>(plan, tmQ, tmX, prm, st);
+    case 6: return launch_one<6, false, stages_for(6), 2>(plan, tmQ, tmX, prm, st);
+    case 7: return launch_one<7, false, stages_for(7), 2>(plan, tmQ, tmX, prm, st);
+    case 8: return launch_one<8, false, stages_for(8), 2>(plan, tmQ, tmX, prm, st);
     default: return cudaErrorInvalidValue;
     }
 }

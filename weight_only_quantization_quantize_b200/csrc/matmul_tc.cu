@@ -45,6 +45,7 @@ struct Params {
     __half *Y;
     int32_t *status;
     int M, K, N;
+    UnpackConsts uk;
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ dequant
         const int tid = threadIdx.x - 64;  // 0..127
+        const UnpackConsts uk = p.uk;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             const int st = kb % kStages;
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int r = 0; r < 8; ++r) {
                     const uint32_t w = reinterpret_cast<const uint32_t *>(q + r * (kBN * 4))[n];
                     uint32_t d[4];
-                    unpack_minus_zero(w, za, zb, d);
+                    unpack_minus_zero(w, za, zb, d, uk);
                     uint32_t o[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -316,7 +318,7 @@ cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensor
                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                       int32_t *status, cudaStream_t st)
 {
-    Params prm{scales, zeros, Y, status, M, K, N};
+    Params prm{scales, zeros, Y, status, M, K, N, unpack_consts()};
     dim3 grid(plan.n_tiles, plan.m_tiles);
     tc_kernel<<<grid, kThreads, plan.smem, st>>>(tmA, tmQ, prm);
     return cudaGetLastError();
