@@ -188,6 +188,28 @@ __device__ __forceinline__ void cluster_sync_all()
                      : "memory");
 }
 
+// Split cluster barrier: arrive (release) now, wait (acquire) later.
+__device__ __forceinline__ void cluster_arrive_release()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Asynchronous 16-byte store into another CTA's shared memory (cluster
+// addresses from mapa); its bytes complete transactions on that CTA's mbarrier.
+__device__ __forceinline__ void st_async_f4(uint32_t remote_addr, float4 v, uint32_t remote_bar)
+{
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            remote_addr),
+        "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar)
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank)
 {
     uint32_t r;

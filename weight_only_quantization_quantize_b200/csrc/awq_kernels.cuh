@@ -22,6 +22,7 @@ struct GemvPlan {
     int stages;
     int xpro_bytes;
     int gmeta_bytes;
+    int recv_bytes;
     size_t smem;
 };
 bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *plan);

@@ -25,8 +25,10 @@
 //                   even-form and four odd-form f16x2 operands with LOP3 only
 //                   and feeds mma.sync m16n8k16 in swap-AB form (columns are
 //                   MMA rows, tokens MMA columns).
-//   epilogue        per-warp partials -> shared memory -> reduced across the
-//                   cluster through distributed shared memory in rank order.
+//   epilogue        each CTA pushes its partial columns into the shared memory
+//                   of the cluster CTA that owns them (st.async, completion as
+//                   transaction bytes on the owner's mbarrier); owners sum the
+//                   K-split partials locally in fixed rank order and write Y.
 #include "awq_kernels.cuh"
 
 namespace awq {
@@ -36,7 +38,6 @@ namespace {
 constexpr int kBN = 128;
 constexpr int kQStage = 4 * 2048;
 constexpr int kStageBytes = 9216;  // 8 KB words + 256 B steps + 64 B zero words, padded
-constexpr int kRedPitch = 132;
 constexpr int kSmemOptIn = 232448;
 
 struct GemvParams {
@@ -49,6 +50,7 @@ struct GemvParams {
     int M, K, N, G, splits;
     int xpro_bytes;   // X' buffer: M * chunks * 16
     int gmeta_bytes;  // per (token, group, half): {1024 S0 + 64 S1, S0 + S1}
+    int recv_bytes;   // partials pushed to this CTA: [src rank][k half][8 tokens][128 / splits]
     // Unpack constants, passed at run time: as compile-time literals the
     // compiler re-materializes them before every use (a LOP3 encodes only one
     // 32-bit immediate), which nearly doubles the integer-pipe work per weight.
@@ -87,17 +89,24 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 
     uint8_t *xpro = smem + S * kStageBytes;
     float2 *gmeta = reinterpret_cast<float2 *>(xpro + p.xpro_bytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.xpro_bytes + p.gmeta_bytes);
+    float *recv = reinterpret_cast<float *>(xpro + p.xpro_bytes + p.gmeta_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.xpro_bytes + p.gmeta_bytes + p.recv_bytes);
     uint64_t *empty = full + S;
+    uint64_t *recv_bar = empty + S;
+    const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(&full[i], 1 + 32);
             mbar_init(&empty[i], kConsumers);
         }
+        mbar_init(recv_bar, 1);
         fence_barrier_init();
+        // expect every rank's partials for the columns this CTA owns
+        mbar_arrive_expect_tx(recv_bar, KH * p.M * cpo * p.splits * 4);
     }
     __syncthreads();
+    cluster_arrive_release();  // barriers initialized; waited on before the first push
 
     float acc[2][4];
 #pragma unroll
@@ -107,14 +116,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 
     if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            const int npf = ng < 64 ? ng : 64;
-            for (int it = 0; it < npf; ++it)
-#pragma unroll
-                for (int w = 0; w < 4; ++w)
-                    tma_prefetch_l2_2d(&tmQ, n0 + 32 * w, (g_begin + it) * 16);
-        }
+        if (lane == 0) prefetch_tmap(&tmQ);
         pdl_wait();
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
@@ -279,40 +281,49 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     }
 
     // ---------------------------------------------------------------- epilogue
-    __syncthreads();
-    float *red = reinterpret_cast<float *>(smem);  // [khalf][token 0..7][column]
-    constexpr int kHalfStride = 8 * kRedPitch;
+    // Push: a consumer thread holds 4 consecutive columns (one 8-column chunk)
+    // for tokens 2t, 2t+1; the chunk's owner is rank chunk % splits.
+    cluster_wait_acquire();  // every CTA of the cluster has initialized its barriers
     if (warp < kConsumers) {
         const int gq = lane >> 2, t = lane & 3;
         const int colw = 32 * (warp & 3) + 4 * gq;
-        float *rh = red + (warp >> 2) * kHalfStride;
+        const int khalf = warp >> 2;
+        const int chunk = colw >> 3;
+        const uint32_t owner = static_cast<uint32_t>(chunk % p.splits);
+        const int lc = (chunk / p.splits) * 8 + (colw & 7);
+        const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile) {
-            const int tok = 2 * t;
-            const int col = colw + 2 * tile;
-            rh[tok * kRedPitch + col] = acc[tile][0];
-            rh[(tok + 1) * kRedPitch + col] = acc[tile][1];
-            rh[tok * kRedPitch + col + 1] = acc[tile][2];
-            rh[(tok + 1) * kRedPitch + col + 1] = acc[tile][3];
+        for (int tk = 0; tk < 2; ++tk) {
+            const int tok = 2 * t + tk;
+            if (tok < p.M) {
+                const float4 v = make_float4(acc[0][tk], acc[0][2 + tk], acc[1][tk], acc[1][2 + tk]);
+                const int off = (((split * KH + khalf) * 8 + tok) * cpo + lc) * 4;
+                st_async_f4(map_to_rank(smem_u32(recv) + off, owner), v, rbar);
+            }
         }
     }
-    cluster_sync_all();
-    const uint32_t red_base = smem_u32(red);
-    for (int e = threadIdx.x; e < p.M * 16; e += kAllThreads) {
-        const int tok = e >> 4;
-        const int ch = e & 15;
-        const int n = n0 + ch * 8;
-        if (ch % p.splits != split || n >= p.N) continue;
+    // Arrive (release: this thread's pushes are performed before it is seen);
+    // the matching wait is the last thing a CTA does, so no CTA exits while a
+    // push from or to it is still in flight, yet nobody idles on it: every CTA
+    // has pushed long before any finishes reducing.
+    cluster_arrive_release();
+    // Reduce the columns this rank owns, partials summed in (rank, k-half) order.
+    if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    const int lchunks = cpo / 8;
+    for (int e = threadIdx.x; e < p.M * lchunks; e += kAllThreads) {
+        const int tok = e / lchunks;
+        const int lch = e - tok * lchunks;
+        const int n = n0 + (lch * p.splits + split) * 8;
+        if (n >= p.N) continue;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.0f;
         for (int r = 0; r < p.splits; ++r) {
 #pragma unroll
             for (int h = 0; h < KH; ++h) {
-                const uint32_t off = red_base + (h * kHalfStride + tok * kRedPitch + ch * 8) * 4;
-                const uint32_t a = map_to_rank(off, r);
-                const float4 lo = ld_cluster_f4(a);
-                const float4 hi = ld_cluster_f4(a + 16);
+                const float4 *src =
+                    reinterpret_cast<const float4 *>(recv + ((r * KH + h) * 8 + tok) * cpo + lch * 8);
+                const float4 lo = src[0], hi = src[1];
                 v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
                 v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
             }
@@ -324,7 +335,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         o.w = __half_as_ushort(__float2half_rn(v[6])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[7]))) << 16);
         *reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(tok) * p.N + n) = o;
     }
-    cluster_sync_all();
+    cluster_wait_acquire();
 }
 
 template <int S, int KH>
@@ -381,37 +392,43 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     const int max_split = G < 8 ? G : 8;
     pl->n_tiles = (N + kBN - 1) / kBN;
     pl->kh = 1;
-    // Measured on the decode shapes: split K until there are about six CTAs
-    // per SM (splits dividing the group count); with four or more CTAs per SM
-    // a 4-deep ring keeps enough bytes in flight, below that 8 stages do.
-    int splits = max_split;
-    for (int sp = 1; sp <= max_split; ++sp) {
-        if (pl->n_tiles * sp >= 6 * num_sms && (G % sp == 0)) {
-            splits = sp;
-            break;
-        }
+    // splits is a power of two so each cluster rank owns 128 / splits columns.
+    // Measured on the decode shapes (K 4096..14336, N 4096..28672): with at
+    // most one 128-column tile per SM, an 8-deep ring and the largest split
+    // that still fits one wave at two CTAs per SM; with more tiles than SMs,
+    // a 4-deep ring and splits up to about six CTAs per SM for load balance.
+    int max_pow2 = 1;
+    while (max_pow2 * 2 <= max_split) max_pow2 *= 2;
+    int splits = 1;
+    if (pl->n_tiles <= num_sms) {
+        pl->stages = 8;
+        while (splits * 2 <= max_pow2 && pl->n_tiles * splits * 2 <= 2 * num_sms) splits *= 2;
+    } else {
+        pl->stages = 4;
+        while (splits * 2 <= max_pow2 && pl->n_tiles * splits < 6 * num_sms) splits *= 2;
     }
-    pl->stages = pl->n_tiles * splits >= 4 * num_sms ? 4 : 8;
 #ifdef AWQ_TUNING
     splits = tune_env("AWQ_TUNE_SPLITS", splits);
-    if (splits > max_split) splits = max_split;
+    if (splits > max_pow2) splits = max_pow2;
     if (splits < 1) splits = 1;
+    while (splits & (splits - 1)) --splits;
     pl->kh = tune_env("AWQ_TUNE_KH", pl->kh);
     pl->stages = tune_env("AWQ_TUNE_STAGES", pl->stages) <= 4 ? 4 : 8;
 #endif
     // X' and the group sums live in shared memory: M * (groups per CTA) * 256 B
     // (+ 8 B per group half); find the smallest split at or above the choice that fits
-    for (; splits <= max_split; ++splits) {
+    for (; splits <= max_pow2; splits *= 2) {
         const int gmax = (G + splits - 1) / splits;
         if (static_cast<size_t>(M) * gmax * (256 + 8 * pl->kh) <= 64 * 1024) break;
     }
-    if (splits > max_split) return false;
+    if (splits > max_pow2) return false;
     pl->splits = splits;
     const int gmax = (G + splits - 1) / splits;
     pl->xpro_bytes = M * gmax * 256;
     pl->gmeta_bytes = (M * gmax * pl->kh * 8 + 15) & ~15;
+    pl->recv_bytes = pl->kh * 8 * kBN * 4;
     pl->smem = 1024 + static_cast<size_t>(pl->stages) * kStageBytes + pl->xpro_bytes + pl->gmeta_bytes +
-               2 * pl->stages * sizeof(uint64_t);
+               pl->recv_bytes + (2 * pl->stages + 1) * sizeof(uint64_t);
     return true;
 }
 
@@ -433,6 +450,7 @@ cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __ha
     prm.splits = plan.splits;
     prm.xpro_bytes = plan.xpro_bytes;
     prm.gmeta_bytes = plan.gmeta_bytes;
+    prm.recv_bytes = plan.recv_bytes;
     prm.mask_lo = 0x000F000Fu;
     prm.mask_hi = 0x00F000F0u;
     prm.magic = 0x64006400u;
