@@ -102,8 +102,8 @@ bool matmul_shape_ok(int64_t M, int64_t K, int64_t N)
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// X / s (binary16, pair-permuted) lives in the workspace unless the
-// small-batch kernel computes it in shared memory itself (M = 1 always does).
+// X / s (binary16, pair-permuted) lives in the workspace, except for M = 1:
+// the decode GEMV computes it in shared memory itself, for every legal K.
 size_t workspace_bytes(int64_t M, int64_t K) { return M == 1 ? 0 : round_up(static_cast<size_t>(2 * M * K), 256); }
 
 awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
@@ -143,16 +143,12 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;
-        if (!plan.prologue) {
-            if (!Xp) return AWQ_ERR_WORKSPACE;
-            if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
-                           static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
-                return AWQ_ERR_CUDA;
-            e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
-            if (e != AWQ_OK) return e;
-        } else {
-            tmX = tmQ;  // unused by the kernel
-        }
+        if (!Xp) return AWQ_ERR_WORKSPACE;
+        if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
+                       static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
+            return AWQ_ERR_CUDA;
+        e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
+        if (e != AWQ_OK) return e;
         return from_cuda(awq::launch_small_m(plan, tmQ, tmX, hX, hs, hsc, zeros, hY, m, k, n,
                                              dev_status, st));
     }

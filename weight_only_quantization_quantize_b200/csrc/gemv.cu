@@ -419,7 +419,7 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     // (+ 8 B per group half); find the smallest split at or above the choice that fits
     for (; splits <= max_pow2; splits *= 2) {
         const int gmax = (G + splits - 1) / splits;
-        if (static_cast<size_t>(M) * gmax * (256 + 8 * pl->kh) <= 64 * 1024) break;
+        if (static_cast<size_t>(M) * gmax * (256 + 8 * pl->kh) <= 80 * 1024) break;
     }
     if (splits > max_pow2) return false;
     pl->splits = splits;

@@ -7,28 +7,26 @@
 // "Group Size Configuration" / "Zero-Point Quantization" (4-bit codes, group
 // 128, zero point).
 //
-// Design (B200):
+// Design (B200), for 1 <= M < 64 tokens (the single-token GEMV with small K
+// uses gemv.cu instead):
 //  * Weights stream once from HBM: a producer warp issues TMA tile loads of
 //    the packed words (one 16-row x 32-column box per consumer warp, 128-byte
-//    swizzled so the consumers' 16-byte shared loads are conflict free) plus
-//    cp.async copies of the group's scales and zero points into a ring of
-//    mbarrier-guarded stages; one stage is one 128-row group.
-//  * Four consumer warps each own 32 output columns.  A lane unpacks one
-//    16-byte load (4 columns x 8 consecutive k) into exact (q - z) binary16
-//    pairs with integer ops and two f16x2 instructions per pair, and feeds
-//    them straight from registers to mma.sync m16n8k16 (fp32 accumulate) in
-//    swap-AB form: the output columns are the MMA rows, the tokens its 8
-//    columns.  The contraction order inside each 8-k word is permuted
-//    (k pairs (0,4),(1,5),(2,6),(3,7)); X / s is stored with the same
-//    permutation, so the sum is unchanged.
-//  * The MMA gives each group's partial sum_k x'_k (q_k - z) in fp32; the
-//    group step is applied once per group (distributivity), y += step * part.
-//  * Split-K across the CTAs of a thread-block cluster; the partial tiles are
-//    reduced through distributed shared memory in a fixed rank order
-//    (deterministic), each rank finishing a slice of the columns.
-//  * X / s: for M <= 8 each CTA computes it for its own k range into shared
-//    memory (no workspace, no extra launch); otherwise a pre-pass writes it
-//    once to the workspace and the producer TMA-loads it per stage.
+//    swizzled so the consumers' 16-byte shared loads are conflict free), of the
+//    group's X / s rows (written once by a pre-pass), plus cp.async copies of
+//    the group's scales and zero points, into a ring of mbarrier-guarded
+//    stages; one stage is one 128-row group.
+//  * Four consumer warps each own 32 output columns.  A lane turns one 16-byte
+//    load (4 columns x 8 consecutive k) into binary16 (q - z) * step values
+//    (two LOP3 masks + f16x2 ops per pair, the step applied in binary16 as in
+//    the tensor-core GEMM) and feeds them from registers to mma.sync m16n8k16
+//    (fp32 accumulate) in swap-AB form: output columns are the MMA rows, the
+//    M tokens (up to 8 tiles of 8) its columns.  The contraction order inside
+//    each 8-k word is permuted (pairs (0,4),(1,5),(2,6),(3,7)); X / s is stored
+//    with the same permutation.
+//  * Split-K across the CTAs of a thread-block cluster; each CTA pushes its
+//    partial columns into the shared memory of the rank that owns them
+//    (st.async, completion counted on the owner's mbarrier) and the owner sums
+//    them in rank order (deterministic).
 #include "awq_kernels.cuh"
 
 namespace awq {
@@ -38,11 +36,8 @@ namespace {
 constexpr int kBN = 128;            // output columns per CTA
 constexpr int kQStage = 4 * 2048;   // 4 boxes of [16 rows x 32 words]
 constexpr int kMetaBytes = 256 + 64;  // 128 scales + 16 zero words
-constexpr int kRedPitch = 132;      // floats per token row of the reduction tile
-constexpr size_t kPrologueMax = 64 * 1024;
 constexpr int kSmemOptIn = 232448;  // 227 KB, the per-block opt-in maximum
 
-constexpr int stages_for(int mt) { return mt <= 2 ? 8 : 4; }
 
 struct Params {
     const __half *X;
@@ -52,9 +47,9 @@ struct Params {
     __half *Y;
     int32_t *status;
     int M, K, N, G, splits;
-    int xbox;          // bytes reserved per staged X' box (0 with the prologue)
+    int xbox;          // bytes reserved per staged X' box
     int stage_bytes;
-    int prologue_bytes;
+    int recv_bytes;    // partials pushed to this CTA: [src rank][8 * MT tokens][128 / splits]
     UnpackConsts uk;
 };
 
@@ -95,18 +90,13 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// KH = warps per 32-column slab: with KH = 2 a warp pair splits each group's
-// 128 rows (k 0..63 and 64..127), doubling the warps that hide MMA and
-// shared-memory latency; the halves are summed in the epilogue.
-template <int MT, bool PRO, int S, int KH>
-__global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
+template <int MT, int S>
+__global__ void __launch_bounds__(160, 1)
     small_m_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmX,
                    const Params p)
 {
-    constexpr int kConsumers = 4 * KH;
-    constexpr int kCThreads = 32 * kConsumers;
-    constexpr int kAllThreads = kCThreads + 32;
-    constexpr int kSteps = 4 / KH;  // 32-row steps per warp per group
+    constexpr int kConsumers = 4;
+    constexpr int kAllThreads = 160;
 
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *smem = align1024(smem_dyn);
@@ -117,23 +107,26 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     const int g_begin = static_cast<int>(static_cast<int64_t>(split) * p.G / p.splits);
     const int g_end = static_cast<int>(static_cast<int64_t>(split + 1) * p.G / p.splits);
     const int ng = g_end - g_begin;
-    const int chunks = ng * 16;  // 8-channel chunks of this CTA's k range
+    const int cpo = kBN / p.splits;
 
-    // the next kernel on the stream may begin its own prologue now
     pdl_launch_dependents();
 
-    uint8_t *xpro = smem + S * p.stage_bytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.prologue_bytes);
+    float *recv = reinterpret_cast<float *>(smem + S * p.stage_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes + p.recv_bytes);
     uint64_t *empty = full + S;
+    uint64_t *recv_bar = empty + S;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1 + 32);     // expect_tx arrival + 32 cp.async arrivals
-            mbar_init(&empty[i], kConsumers);  // one per consumer warp
+            mbar_init(&full[i], 1 + 32);  // expect_tx arrival + 32 cp.async arrivals
+            mbar_init(&empty[i], kConsumers);
         }
+        mbar_init(recv_bar, 1);
         fence_barrier_init();
+        mbar_arrive_expect_tx(recv_bar, p.M * cpo * p.splits * 4);
     }
     __syncthreads();
+    cluster_arrive_release();
 
     float acc[2][MT][4];
 #pragma unroll
@@ -147,17 +140,10 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
-            if (!PRO) prefetch_tmap(&tmX);
-            // Warm L2 with this CTA's packed weights while the previous kernel
-            // on the stream finishes; the real loads below come after the wait.
-            const int npf = ng < 64 ? ng : 64;
-            for (int it = 0; it < npf; ++it)
-#pragma unroll
-                for (int w = 0; w < 4; ++w)
-                    tma_prefetch_l2_2d(&tmQ, n0 + 32 * w, (g_begin + it) * 16);
+            prefetch_tmap(&tmX);
         }
         pdl_wait();
-        const uint32_t tx = kQStage + (PRO ? 0 : 2 * p.M * 128);
+        const uint32_t tx = kQStage + 2 * p.M * 128;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
             const int st = it % S;
@@ -172,10 +158,8 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
                     tma_load_2d(stg + w * 2048, &tmQ, &full[st], n0 + 32 * w, g * 16);
-                if (!PRO) {
-                    tma_load_2d(stg + kQStage, &tmX, &full[st], g * kGroup, 0);
-                    tma_load_2d(stg + kQStage + p.xbox, &tmX, &full[st], g * kGroup + 64, 0);
-                }
+                tma_load_2d(stg + kQStage, &tmX, &full[st], g * kGroup, 0);
+                tma_load_2d(stg + kQStage + p.xbox, &tmX, &full[st], g * kGroup + 64, 0);
             }
             uint8_t *meta = stg + kQStage + 2 * p.xbox;
             if (lane < 16) {
@@ -196,24 +180,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         // ------------------------------------------------------------ consumers
         const int gq = lane >> 2;
         const int t = lane & 3;
-        const int slab = warp & 3;
-        const int khalf = warp >> 2;            // 0 when KH == 1
-        const int colw = 32 * slab + 4 * gq;    // my 4 columns: colw .. colw+3 (tile-local)
-        pdl_wait();
-        if (PRO) {
-            const int total = p.M * chunks;
-            for (int idx = threadIdx.x; idx < total; idx += kCThreads) {
-                const int tok = idx / chunks;
-                const int ch = idx - tok * chunks;
-                const int k = g_begin * kGroup + ch * 8;
-                const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(tok) * p.K + k));
-                const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(p.s + k));
-                *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok) * chunks + (ch ^ (tok & 7))) * 16) =
-                    prescale8(xv, sv);
-            }
-            named_bar_sync(1, kCThreads);
-        }
-        const uint32_t xpro_base = smem_u32(xpro);
+        const int colw = 32 * warp + 4 * gq;  // my 4 columns: colw .. colw+3 (tile-local)
         const UnpackConsts uk = p.uk;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
@@ -227,133 +194,96 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
             const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
             const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
             const int zsh = (colw & 7) * 4;
-            uint32_t za[4], zb[4];
+            uint32_t za[4], zb[4], st2[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) zero_constants((zw >> (zsh + 4 * c)) & 15u, za[c], zb[c]);
-
-            // with few token tiles, two accumulator sets (even / odd step) halve the
-            // MMA dependency chains; more token tiles already give independent chains
-            constexpr int kSets = MT <= 2 ? 2 : 1;
-            float grp[kSets][2][MT][4];
+            {
+                const uint32_t s01 = sc.x, s23 = sc.y;
+                st2[0] = (s01 & 0xFFFFu) * 0x10001u;
+                st2[1] = (s01 >> 16) * 0x10001u;
+                st2[2] = (s23 & 0xFFFFu) * 0x10001u;
+                st2[3] = (s23 >> 16) * 0x10001u;
+            }
+            const uint8_t *qslab = stg + warp * 2048;
+            const uint8_t *xstage = stg + kQStage;
 #pragma unroll
-            for (int b = 0; b < kSets; ++b)
-#pragma unroll
-                for (int a = 0; a < 2; ++a)
-#pragma unroll
-                    for (int j = 0; j < MT; ++j)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) grp[b][a][j][i] = 0.0f;
-
-            const uint32_t qslab = smem_u32(stg) + slab * 2048;
-            const uint32_t xstage = smem_u32(stg) + kQStage;
-#pragma unroll
-            for (int ss = 0; ss < kSteps; ++ss) {
-                const int sidx = khalf * kSteps + ss;
+            for (int sidx = 0; sidx < 4; ++sidx) {
                 const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);  // packed row in the group
-                const uint4 wq = lds128(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
-                uint32_t bx[MT][4];
+                const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
+                uint4 bx[MT];
 #pragma unroll
                 for (int j = 0; j < MT; ++j) {
                     const int tok = 8 * j + gq;
-                    if (tok < p.M) {
-                        uint32_t addr;
-                        if (PRO)
-                            addr = xpro_base + ((tok * chunks) + ((it * 16 + r) ^ (tok & 7))) * 16;
-                        else
-                            addr = xstage + (sidx >> 1) * p.xbox + tok * 128 + (((r & 7) ^ (tok & 7)) << 4);
-                        const uint4 v = lds128(addr);
-                        bx[j][0] = v.x;
-                        bx[j][1] = v.y;
-                        bx[j][2] = v.z;
-                        bx[j][3] = v.w;
-                    } else {
-                        bx[j][0] = bx[j][1] = bx[j][2] = bx[j][3] = 0u;
-                    }
+                    bx[j] = make_uint4(0u, 0u, 0u, 0u);
+                    if (tok < p.M)
+                        bx[j] = *reinterpret_cast<const uint4 *>(xstage + (sidx >> 1) * p.xbox + tok * 128 +
+                                                                 (((r & 7) ^ (tok & 7)) << 4));
                 }
+                const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
                 uint32_t d[4][4];
-                unpack_minus_zero(wq.x, za[0], zb[0], d[0], uk);
-                unpack_minus_zero(wq.y, za[1], zb[1], d[1], uk);
-                unpack_minus_zero(wq.z, za[2], zb[2], d[2], uk);
-                unpack_minus_zero(wq.w, za[3], zb[3], d[3], uk);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t e[4];
+                    unpack_minus_zero(w[c], za[c], zb[c], e, uk);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d[c][i]) : "r"(e[i]), "r"(st2[c]));
+                }
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
-                    const uint32_t a0[4] = {d[2 * tile][0], d[2 * tile + 1][0], d[2 * tile][1],
-                                            d[2 * tile + 1][1]};
-                    const uint32_t a1[4] = {d[2 * tile][2], d[2 * tile + 1][2], d[2 * tile][3],
-                                            d[2 * tile + 1][3]};
+                    const uint32_t a0[4] = {d[2 * tile][0], d[2 * tile + 1][0], d[2 * tile][1], d[2 * tile + 1][1]};
+                    const uint32_t a1[4] = {d[2 * tile][2], d[2 * tile + 1][2], d[2 * tile][3], d[2 * tile + 1][3]};
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
-                        mma_16816(grp[ss % kSets][tile][j], a0, bx[j][0], bx[j][1]);
-                        mma_16816(grp[ss % kSets][tile][j], a1, bx[j][2], bx[j][3]);
+                        mma_16816(acc[tile][j], a0, bx[j].x, bx[j].y);
+                        mma_16816(acc[tile][j], a1, bx[j].z, bx[j].w);
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
-            const float2 s01 = __half22float2(*reinterpret_cast<const __half2 *>(&sc.x));
-            const float2 s23 = __half22float2(*reinterpret_cast<const __half2 *>(&sc.y));
-#pragma unroll
-            for (int j = 0; j < MT; ++j) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float f0 = i < 2 ? s01.x : s01.y;
-                    const float f1 = i < 2 ? s23.x : s23.y;
-                    float p0 = grp[0][0][j][i], p1 = grp[0][1][j][i];
-                    if (kSets == 2) {
-                        p0 += grp[kSets - 1][0][j][i];
-                        p1 += grp[kSets - 1][1][j][i];
-                    }
-                    acc[0][j][i] = fmaf(f0, p0, acc[0][j][i]);
-                    acc[1][j][i] = fmaf(f1, p1, acc[1][j][i]);
-                }
-            }
         }
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     }
 
     // ---------------------------------------------------------------- epilogue
-    __syncthreads();  // every stage consumed: the ring can hold the partial tiles
-    // red[khalf][token][column]
-    float *red = reinterpret_cast<float *>(smem);
-    constexpr int kHalfStride = 8 * MT * kRedPitch;
+    // Push: a consumer thread holds columns colw .. colw+3 (one 8-column chunk)
+    // for tokens 8j + 2t, 8j + 2t + 1; the chunk's owner is rank chunk % splits.
+    cluster_wait_acquire();
     if (warp < kConsumers) {
         const int gq = lane >> 2, t = lane & 3;
-        const int colw = 32 * (warp & 3) + 4 * gq;
-        float *rh = red + (warp >> 2) * kHalfStride;
+        const int colw = 32 * warp + 4 * gq;
+        const int chunk = colw >> 3;
+        const uint32_t owner = static_cast<uint32_t>(chunk % p.splits);
+        const int lc = (chunk / p.splits) * 8 + (colw & 7);
+        const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile)
+        for (int j = 0; j < MT; ++j)
 #pragma unroll
-            for (int j = 0; j < MT; ++j) {
-                const int tok = 8 * j + 2 * t;
-                const int col = colw + 2 * tile;
-                rh[tok * kRedPitch + col] = acc[tile][j][0];
-                rh[(tok + 1) * kRedPitch + col] = acc[tile][j][1];
-                rh[tok * kRedPitch + col + 1] = acc[tile][j][2];
-                rh[(tok + 1) * kRedPitch + col + 1] = acc[tile][j][3];
+            for (int tk = 0; tk < 2; ++tk) {
+                const int tok = 8 * j + 2 * t + tk;
+                if (tok < p.M) {
+                    const float4 v = make_float4(acc[0][j][tk], acc[0][j][2 + tk], acc[1][j][tk], acc[1][j][2 + tk]);
+                    const int off = ((split * 8 * MT + tok) * cpo + lc) * 4;
+                    st_async_f4(map_to_rank(smem_u32(recv) + off, owner), v, rbar);
+                }
             }
     }
-    cluster_sync_all();
-    // this rank finishes the 8-column chunks ch with ch % splits == rank,
-    // summing the partials in (rank, k-half) order
-    const uint32_t red_base = smem_u32(red);
-    for (int e = threadIdx.x; e < p.M * 16; e += kAllThreads) {
-        const int tok = e >> 4;
-        const int ch = e & 15;
-        const int n = n0 + ch * 8;
-        if (ch % p.splits != split || n >= p.N) continue;
+    cluster_arrive_release();  // pushes performed before the final wait completes anywhere
+    if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    const int lchunks = cpo / 8;
+    for (int e = threadIdx.x; e < p.M * lchunks; e += kAllThreads) {
+        const int tok = e / lchunks;
+        const int lch = e - tok * lchunks;
+        const int n = n0 + (lch * p.splits + split) * 8;
+        if (n >= p.N) continue;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.0f;
         for (int r = 0; r < p.splits; ++r) {
-#pragma unroll
-            for (int h = 0; h < KH; ++h) {
-                const uint32_t off = red_base + (h * kHalfStride + tok * kRedPitch + ch * 8) * 4;
-                const uint32_t a = map_to_rank(off, r);
-                const float4 lo = ld_cluster_f4(a);
-                const float4 hi = ld_cluster_f4(a + 16);
-                v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
-                v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
-            }
+            const float4 *src = reinterpret_cast<const float4 *>(recv + ((r * 8 * MT) + tok) * cpo + lch * 8);
+            const float4 lo = src[0], hi = src[1];
+            v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+            v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
         }
         uint4 o;
         o.x = __half_as_ushort(__float2half_rn(v[0])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
@@ -362,17 +292,16 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         o.w = __half_as_ushort(__float2half_rn(v[6])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[7]))) << 16);
         *reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(tok) * p.N + n) = o;
     }
-    cluster_sync_all();  // keep this CTA's partials alive until every rank has read them
+    cluster_wait_acquire();
 }
 
-template <int MT, bool PRO, int S, int KH>
+template <int MT, int S>
 cudaError_t launch_one(const SmallMPlan &plan, const CUtensorMap &tmQ, const CUtensorMap &tmX,
                        const Params &prm, cudaStream_t st)
 {
-    auto kern = small_m_kernel<MT, PRO, S, KH>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.splits, plan.n_tiles, 1);
-    cfg.blockDim = dim3(32 * (4 * KH + 1), 1, 1);
+    cfg.blockDim = dim3(160, 1, 1);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -384,30 +313,33 @@ cudaError_t launch_one(const SmallMPlan &plan, const CUtensorMap &tmQ, const CUt
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, tmQ, tmX, prm);
+    return cudaLaunchKernelEx(&cfg, small_m_kernel<MT, S>, tmQ, tmX, prm);
 }
 
-template <int MT, bool PRO, int S, int KH>
+template <int MT, int S>
 cudaError_t configure_one()
 {
-    return cudaFuncSetAttribute(small_m_kernel<MT, PRO, S, KH>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemOptIn);
+    return cudaFuncSetAttribute(small_m_kernel<MT, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemOptIn);
+}
+
+int stage_bytes_for(int M)
+{
+    const int xbox = (M * 128 + 1023) & ~1023;
+    return (kQStage + 2 * xbox + kMetaBytes + 1023) & ~1023;
 }
 
 }  // namespace
 
 cudaError_t configure_small_m()
 {
-    cudaError_t e = cudaSuccess;
-    const cudaError_t r[] = {
-        configure_one<1, true, stages_for(1), 2>(),  configure_one<1, true, stages_for(1), 1>(),
-        configure_one<1, false, stages_for(1), 2>(), configure_one<2, false, stages_for(2), 2>(),
-        configure_one<3, false, stages_for(3), 2>(), configure_one<4, false, stages_for(4), 2>(),
-        configure_one<5, false, stages_for(5), 2>(), configure_one<6, false, stages_for(6), 2>(),
-        configure_one<7, false, stages_for(7), 2>(), configure_one<8, false, stages_for(8), 2>()};
+    const cudaError_t r[] = {configure_one<1, 8>(), configure_one<1, 4>(), configure_one<2, 8>(),
+                             configure_one<2, 4>(), configure_one<3, 4>(), configure_one<4, 4>(),
+                             configure_one<5, 4>(), configure_one<6, 4>(), configure_one<7, 4>(),
+                             configure_one<8, 4>()};
     for (cudaError_t x : r)
-        if (x != cudaSuccess) e = x;
-    return e;
+        if (x != cudaSuccess) return x;
+    return cudaSuccess;
 }
 
 #ifdef AWQ_TUNING
@@ -423,44 +355,27 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
     SmallMPlan pl{};
     pl.mt = (M + 7) / 8;
     pl.n_tiles = (N + kBN - 1) / kBN;
-    pl.stages = stages_for(pl.mt);
-    pl.kh = 2;
+    pl.prologue = false;
+    pl.kh = 1;
+    pl.stages = pl.mt <= 2 ? 8 : 4;
     const int G = K / kGroup;
-    const int max_split = G < 8 ? G : 8;
-    const int target = 2 * num_sms;
-    int splits = max_split;
-    for (int sp = 1; sp <= max_split; ++sp) {
-        if (pl.n_tiles * sp >= target && (G % sp == 0)) {
-            splits = sp;
-            break;
-        }
-    }
+    int max_pow2 = 1;
+    while (max_pow2 * 2 <= 8 && max_pow2 * 2 <= G) max_pow2 *= 2;
+    const int stage_bytes = stage_bytes_for(M);
+    const int recv_bytes = 8 * pl.mt * kBN * 4;
+    size_t smem = 1024 + static_cast<size_t>(pl.stages) * stage_bytes + recv_bytes + (2 * pl.stages + 1) * 8;
+    const int per_sm = static_cast<int>(228 * 1024 / (smem + 1024));
+    // one wave: the largest power-of-two split with n_tiles * splits <= CTAs resident
+    int splits = 1;
+    while (splits * 2 <= max_pow2 && pl.n_tiles * splits * 2 <= (per_sm < 1 ? 1 : per_sm) * num_sms) splits *= 2;
 #ifdef AWQ_TUNING
     splits = tune_env("AWQ_TUNE_SPLITS", splits);
-    if (splits > max_split) splits = max_split;
+    if (splits > max_pow2) splits = max_pow2;
     if (splits < 1) splits = 1;
-    if (pl.mt == 1) pl.kh = tune_env("AWQ_TUNE_KH", pl.kh);
+    while (splits & (splits - 1)) --splits;
 #endif
-    pl.prologue = false;
-    if (pl.mt == 1) {
-        // X / s in shared memory needs M * (groups per split) * 256 bytes
-        for (int sp = splits; sp <= max_split; ++sp) {
-            const int gmax = (G + sp - 1) / sp;
-            if (static_cast<size_t>(M) * gmax * 256 <= kPrologueMax) {
-                pl.prologue = true;
-                splits = sp;
-                break;
-            }
-        }
-    }
-    if (!pl.prologue) pl.kh = 2;
     pl.splits = splits;
-    const int xbox = pl.prologue ? 0 : ((M * 128 + 1023) & ~1023);
-    const int stage_bytes = (kQStage + 2 * xbox + kMetaBytes + 1023) & ~1023;
-    const int gmax = (G + splits - 1) / splits;
-    const size_t pro = pl.prologue ? static_cast<size_t>(M) * gmax * 256 : 0;
-    pl.smem = 1024 /* alignment slack */ + static_cast<size_t>(pl.stages) * stage_bytes + pro +
-              2 * pl.stages * sizeof(uint64_t);
+    pl.smem = smem;
     return pl;
 }
 
@@ -498,24 +413,20 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
     prm.N = N;
     prm.G = K / kGroup;
     prm.splits = plan.splits;
-    prm.xbox = plan.prologue ? 0 : ((M * 128 + 1023) & ~1023);
-    prm.stage_bytes = (kQStage + 2 * prm.xbox + kMetaBytes + 1023) & ~1023;
-    const int gmax = (prm.G + plan.splits - 1) / plan.splits;
-    prm.prologue_bytes = plan.prologue ? M * gmax * 256 : 0;
+    prm.xbox = (M * 128 + 1023) & ~1023;
+    prm.stage_bytes = stage_bytes_for(M);
+    prm.recv_bytes = 8 * plan.mt * kBN * 4;
     prm.uk = unpack_consts();
+    const bool deep = plan.stages == 8;
     switch (plan.mt) {
-    case 1:
-        if (plan.prologue)
-            return plan.kh == 1 ? launch_one<1, true, stages_for(1), 1>(plan, tmQ, tmX, prm, st)
-                                : launch_one<1, true, stages_for(1), 2>(plan, tmQ, tmX, prm, st);
-        return launch_one<1, false, stages_for(1), 2>(plan, tmQ, tmX, prm, st);
-    case 2: return launch_one<2, false, stages_for(2), 2>(plan, tmQ, tmX, prm, st);
-    case 3: return launch_one<3, false, stages_for(3), 2>(plan, tmQ, tmX, prm, st);
-    case 4: return launch_one<4, false, stages_for(4), 2>(plan, tmQ, tmX, prm, st);
-    case 5: return launch_one<5, false, stages_for(5), 2>(plan, tmQ, tmX, prm, st);
-    case 6: return launch_one<6, false, stages_for(6), 2>(plan, tmQ, tmX, prm, st);
-    case 7: return launch_one<7, false, stages_for(7), 2>(plan, tmQ, tmX, prm, st);
-    case 8: return launch_one<8, false, stages_for(8), 2>(plan, tmQ, tmX, prm, st);
+    case 1: return deep ? launch_one<1, 8>(plan, tmQ, tmX, prm, st) : launch_one<1, 4>(plan, tmQ, tmX, prm, st);
+    case 2: return deep ? launch_one<2, 8>(plan, tmQ, tmX, prm, st) : launch_one<2, 4>(plan, tmQ, tmX, prm, st);
+    case 3: return launch_one<3, 4>(plan, tmQ, tmX, prm, st);
+    case 4: return launch_one<4, 4>(plan, tmQ, tmX, prm, st);
+    case 5: return launch_one<5, 4>(plan, tmQ, tmX, prm, st);
+    case 6: return launch_one<6, 4>(plan, tmQ, tmX, prm, st);
+    case 7: return launch_one<7, 4>(plan, tmQ, tmX, prm, st);
+    case 8: return launch_one<8, 4>(plan, tmQ, tmX, prm, st);
     default: return cudaErrorInvalidValue;
     }
 }
