@@ -22,6 +22,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "awq_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle_awq.so")
+# A pre-built oracle library to load instead (used by the tests that check the
+# pins catch deliberately broken copies of the oracle).
+_LIB_OVERRIDE = os.environ.get("AWQ_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -45,26 +48,33 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library (marshalling only)."""
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.awq_oracle_half_to_double.argtypes = [ctypes.c_uint16]
+    lib.awq_oracle_half_to_double.restype = ctypes.c_double
+    lib.awq_oracle_double_to_half.argtypes = [ctypes.c_double]
+    lib.awq_oracle_double_to_half.restype = ctypes.c_uint16
+    lib.awq_oracle_act_stats.argtypes = [P, I64, I64, P]
+    lib.awq_oracle_compute_scales.argtypes = [P, I64, P]
+    lib.awq_oracle_quantize_pack.argtypes = [P, P, I64, I64, P, P, P]
+    lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
+    lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
+    for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
+              lib.awq_oracle_quantize_pack, lib.awq_oracle_dequant, lib.awq_oracle_matmul):
+        f.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
-            P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-            lib.awq_oracle_half_to_double.argtypes = [ctypes.c_uint16]
-            lib.awq_oracle_half_to_double.restype = ctypes.c_double
-            lib.awq_oracle_double_to_half.argtypes = [ctypes.c_double]
-            lib.awq_oracle_double_to_half.restype = ctypes.c_uint16
-            lib.awq_oracle_act_stats.argtypes = [P, I64, I64, P]
-            lib.awq_oracle_compute_scales.argtypes = [P, I64, P]
-            lib.awq_oracle_quantize_pack.argtypes = [P, P, I64, I64, P, P, P]
-            lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
-            lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
-            for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
-                      lib.awq_oracle_quantize_pack, lib.awq_oracle_dequant, lib.awq_oracle_matmul):
-                f.restype = ctypes.c_int
-            _lib = lib
+            if _LIB_OVERRIDE:
+                _lib = configure(ctypes.CDLL(_LIB_OVERRIDE))
+            else:
+                build()
+                _lib = configure(ctypes.CDLL(_LIB))
     return _lib
 
 

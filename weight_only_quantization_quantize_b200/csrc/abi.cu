@@ -4,6 +4,7 @@
 // one-time per-device architecture check, TMA descriptor encoding, workspace
 // accounting and the choice of tile path.  Every step of the computation runs
 // in the kernels of quantize.cu, matmul_small.cu and matmul_tc.cu.
+#include <cstdlib>
 #include <mutex>
 
 #include "awq_kernels.cuh"
@@ -132,7 +133,11 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
 
     CUtensorMap tmQ, tmX;
     awq::GemvPlan gplan;
-    if (M <= 8 && awq::plan_gemv(m, k, n, sms, &gplan)) {
+    bool use_gemv = M <= 8;
+#ifdef AWQ_TUNING
+    if (getenv("AWQ_TUNE_GEMV_MAXM")) use_gemv = M <= atoi(getenv("AWQ_TUNE_GEMV_MAXM"));
+#endif
+    if (use_gemv && awq::plan_gemv(m, k, n, sms, &gplan)) {
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;

@@ -139,6 +139,19 @@ __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__res
 }
 
 // ------------------------------------------------------------------ quantize_pack
+// rint(fl(w / sf)), the code decision, without a division per weight.
+// y = fl(w * fl(1/sf)) differs from the IEEE quotient by at most
+// |w/sf| * (2^-23 + 2^-24 + 2^-47) < |y| * 2^-21.  Both values round to the same
+// integer whenever y lies farther than that from the nearest tie point k + 1/2;
+// otherwise (rarely) the correctly rounded quotient decides.
+__device__ __forceinline__ int rint_quotient(float w, float sf, float rsf)
+{
+    const float y = __fmul_rn(w, rsf);
+    const float tie = floorf(y) + 0.5f;
+    if (fabsf(y - tie) > fmaf(fabsf(y), 0x1p-21f, 0x1p-60f)) return __float2int_rn(y);
+    return __float2int_rn(__fdiv_rn(w, sf));
+}
+
 // Block = one 128-row group x 256 columns.  Warp w owns rows 16w..16w+15 of
 // the group; lane l owns columns 8l..8l+7, so every row is read as one
 // 512-byte coalesced warp load.  The per-column min/max is reduced across the
@@ -211,7 +224,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half *__rest
     __syncthreads();
     if (!active) return;
 
-    float sf[8];
+    float sf[8], rsf[8];
     int zc[8];
     uint16_t sh[8];
 #pragma unroll
@@ -228,6 +241,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half *__rest
         if ((bits & 0x7FFF) == 0) bits = 1;  // never a zero step
         sh[c] = bits;
         sf[c] = __half2float(__ushort_as_half(bits));
+        rsf[c] = __frcp_rn(sf[c]);
         float zf = rintf(__fdiv_rn(-b, sf[c]));
         zf = fminf(fmaxf(zf, 0.0f), 15.0f);
         zc[c] = static_cast<int>(zf);
@@ -243,7 +257,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const __half *__rest
             for (int j = 0; j < 8; ++j) {
                 const __half *hr = reinterpret_cast<const __half *>(&raw[h * 8 + j]);
                 const float v = __fmul_rn(__half2float(hr[c]), sk[h * 8 + j]);
-                int q = __float2int_rn(__fdiv_rn(v, sf[c])) + zc[c];
+                int q = rint_quotient(v, sf[c], rsf[c]) + zc[c];
                 q = min(max(q, 0), 15);
                 acc |= static_cast<uint32_t>(q) << (4 * j);
             }
