@@ -58,9 +58,10 @@ def test_noalloc_matches_gemm_on_consecutive_calls():
     assert torch.cuda.is_available()
     L = awq.lib()
     stream = P(torch.cuda.current_stream().cuda_stream)
-    # consecutive calls with different problems (small-batch and tcgen05 tile
-    # paths), then the first problem again: stale scratch contents must not leak
-    cases = [(16, 4096, 4096, 1), (200, 2048, 1032, 2), (48, 14336, 1024, 3), (16, 4096, 4096, 1)]
+    # consecutive calls with different problems (decode, small-batch and tcgen05
+    # tile paths), then earlier problems again: stale scratch contents must not leak
+    cases = [(16, 4096, 4096, 1), (200, 2048, 1032, 2), (1, 4096, 6144, 4), (48, 14336, 1024, 3),
+             (2, 14336, 1032, 5), (1, 4096, 6144, 4), (16, 4096, 4096, 1)]
     layers = {}
     for M, K, N, seed in cases:
         if seed not in layers:
