@@ -139,6 +139,29 @@ def test_quantize_pack_bit_exact_small_and_ragged(K, N):
     quantize_both(L.W, s.cpu())
 
 
+def test_quantize_pack_exact_ties_and_clamping():
+    # Every group column spans [-1, 0.875] in multiples of 1/16 (times a
+    # power-of-two scale), so the step is exactly 1/8 of the scale and half of
+    # the quotients w'/step are exact half-integers: the code decision must
+    # break those ties to even exactly as the definition does.  One block of
+    # groups is shifted positive, so its zero point clamps to 0 and its codes
+    # clamp at 15.
+    rng = np.random.default_rng(5)
+    K, N = 512, 1040
+    W = rng.integers(-16, 15, size=(K, N)).astype(np.float32) / 16
+    W[0::128, :] = -1.0
+    W[1::128, :] = 0.875
+    W[128:256, :64] = np.abs(W[128:256, :64]) + 0.5
+    s = np.ones(K, dtype=np.float32)
+    s[256:384] = 2.0
+    s[384:] = 0.5
+    Wh = torch.from_numpy(W).half()
+    sh = torch.from_numpy(s).half()
+    wp = W.astype(np.float64) * s[:, None]
+    assert np.mean(np.abs(wp * 8 / s[:, None] - np.round(wp * 8 / s[:, None]) ) == 0.5) > 0.3  # many exact ties
+    quantize_both(Wh, sh)
+
+
 # ------------------------------------------------------------------ matmul (all tile paths)
 @pytest.mark.parametrize("M", [1, 2, 7, 8, 9, 16, 33, 48, 63, 64, 65, 127, 128, 200, 256])
 @pytest.mark.parametrize("K,N", [(1024, 1024), (1152, 1032), (128, 8), (2048, 264)])

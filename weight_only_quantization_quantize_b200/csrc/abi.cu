@@ -69,7 +69,7 @@ awq_status_t device_ready(int *sms)
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
             if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
-                awq::configure_gemv() != cudaSuccess) {
+                awq::configure_gemv() != cudaSuccess || awq::configure_quantize() != cudaSuccess) {
                 cudaGetLastError();
                 return AWQ_ERR_CUDA;
             }
@@ -259,10 +259,13 @@ awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, 
     int sms = 0;
     awq_status_t e = device_ready(&sms);
     if (e != AWQ_OK) return e;
-    return from_cuda(awq::launch_quantize_pack(
-        reinterpret_cast<const __half *>(W), reinterpret_cast<const __half *>(s), static_cast<int>(K),
-        static_cast<int>(N), Q, reinterpret_cast<__half *>(scales), zeros, dev_status,
-        static_cast<cudaStream_t>(stream)));
+    CUtensorMap tmW;
+    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, N, K, N * 2, 256, kGroup,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return AWQ_ERR_CUDA;
+    return from_cuda(awq::launch_quantize_pack(tmW, reinterpret_cast<const __half *>(s), static_cast<int>(K),
+                                               static_cast<int>(N), Q, reinterpret_cast<__half *>(scales),
+                                               zeros, dev_status, sms, static_cast<cudaStream_t>(stream)));
 }
 
 size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N)

@@ -10,8 +10,9 @@ cudaError_t launch_act_stats(const __half *xcal, int R, int K, float *m, int32_t
                              cudaStream_t st);
 cudaError_t launch_compute_scales(const float *m, int K, uint16_t *s, int32_t *status,
                                   cudaStream_t st);
-cudaError_t launch_quantize_pack(const __half *W, const __half *s, int K, int N, int32_t *Q,
-                                 __half *scales, int32_t *zeros, int32_t *status,
+cudaError_t configure_quantize();
+cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K, int N, int32_t *Q,
+                                 __half *scales, int32_t *zeros, int32_t *status, int num_sms,
                                  cudaStream_t st);
 
 // gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group

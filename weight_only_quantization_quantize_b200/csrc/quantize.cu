@@ -139,148 +139,293 @@ __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__res
 }
 
 // ------------------------------------------------------------------ quantize_pack
-// rint(fl(w / sf)), the code decision, without a division per weight.
-// y = fl(w * fl(1/sf)) differs from the IEEE quotient by at most
-// |w/sf| * (2^-23 + 2^-24 + 2^-47) < |y| * 2^-21.  Both values round to the same
-// integer whenever y lies farther than that from the nearest tie point k + 1/2;
-// otherwise (rarely) the correctly rounded quotient decides.
-__device__ __forceinline__ int rint_quotient(float w, float sf, float rsf)
+// Persistent CTAs (one per SM, 16 warps) walk tiles of one 128-row group x
+// 256 columns; TMA brings each 64 KB tile of W into a two-deep shared-memory
+// ring.  Warp w owns rows 8w..8w+7 (packed row w of the group) and lane l owns
+// columns 8l..8l+7, so every thread reads 8 x 16 bytes and writes one 32-byte
+// run of packed words.
+//   pass 1  w' = w * s_k (exact: an fma of two binary16 into float), column
+//           max / min over the thread's 8 rows (NaN-propagating), then across
+//           the 16 warps in shared memory by one thread per column, which
+//           also derives the column's step, zero point and reciprocal step.
+//   pass 2  the code decision rint(fl(w' / step)) without a division per
+//           weight: y = w' * fl(1 / step) lies within |y| * 2^-23 of the
+//           exact quotient, and adding 1.5 * 2^23 + z rounds y to an integer
+//           in the low mantissa bits (q = those bits, packed by one integer
+//           multiply-add per code).  A code whose y lies within 2^-18 of a
+//           half-integer is redone with the IEEE division, as is every code
+//           of a column whose extreme codes fall outside 0..15 (clamping).
+// Pairs of columns go through the packed float32x2 multiply / add.
+namespace {
+
+constexpr int kQTileN = 256;                     // columns per tile
+constexpr int kQTileBytes = kGroup * kQTileN * 2;  // 64 KB of binary16
+constexpr int kQThreads = 512;                   // 16 warps: one packed row each
+constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u;
+// sum_j kMagicBits * 16^j (mod 2^32): removed once from a word built with
+// one multiply-add per code from the raw bits of magic + code
+constexpr uint32_t kMagicWord = kMagicBits * 0x11111111u;
+constexpr float kTieMargin = 0.5f - 0x1p-18f;
+
+struct QuantParams {
+    const __half *s;
+    int32_t *Q;
+    __half *scales;
+    int32_t *zeros;
+    int32_t *status;
+    int K, N, G, n_ctiles;
+    int tiles;
+};
+
+struct QuantSmem {
+    uint8_t stage[2][kQTileBytes];
+    float red_max[16][kQTileN];
+    float red_min[16][kQTileN];
+    float rsf[kQTileN];   // fl(1 / step)
+    float cmag[kQTileN];  // 1.5 * 2^23 + z
+    float step[kQTileN];  // step as float (exact fallback)
+    int zc[kQTileN];      // zero point | 0x100 when the column needs clamping
+    uint64_t full[2];
+};
+
+__device__ __forceinline__ float fold(uint16_t w, uint16_t sk)
 {
-    const float y = __fmul_rn(w, rsf);
-    const float tie = floorf(y) + 0.5f;
-    if (fabsf(y - tie) > fmaf(fabsf(y), 0x1p-21f, 0x1p-60f)) return __float2int_rn(y);
-    return __float2int_rn(__fdiv_rn(w, sf));
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(w), "h"(sk), "f"(-0.0f));
+    return d;  // w * s_k, exact in float (11 x 11 significant bits)
+}
+__device__ __forceinline__ float fmax_nan(float a, float b)
+{
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ float fmin_nan(float a, float b)
+{
+    float d;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long pk(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk(unsigned long long v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
-// Block = one 128-row group x 256 columns.  Warp w owns rows 16w..16w+15 of
-// the group; lane l owns columns 8l..8l+7, so every row is read as one
-// 512-byte coalesced warp load.  The per-column min/max is reduced across the
-// 8 warps in shared memory, every thread derives (scale, zero) for its 8
-// columns, encodes its 16 x 8 codes and writes two packed rows of 8 words.
-__global__ void __launch_bounds__(256) quantize_pack_kernel(const __half *__restrict__ W,
-                                                           const __half *__restrict__ s, int K,
-                                                           int N, int32_t *__restrict__ Q,
-                                                           __half *__restrict__ scales,
-                                                           int32_t *__restrict__ zeros,
-                                                           int32_t *status)
+// The code decision with the correctly rounded quotient (the definition).
+__device__ __forceinline__ uint32_t code_exact(float wp, float step, int z)
 {
-    __shared__ float red_max[8][256];
-    __shared__ float red_min[8][256];
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int g = blockIdx.y;
-    const int n = blockIdx.x * 256 + lane * 8;
-    const int k0 = g * kGroup + warp * 16;
-    const bool active = n < N;
+    int q = static_cast<int>(rintf(__fdiv_rn(wp, step))) + z;
+    return static_cast<uint32_t>(min(max(q, 0), 15));
+}
 
-    // per-row channel scale (same for every lane: broadcast loads)
-    float sk[16];
-    bool bad = false;
-    {
-        const uint4 s0 = __ldg(reinterpret_cast<const uint4 *>(s + k0));
-        const uint4 s1 = __ldg(reinterpret_cast<const uint4 *>(s + k0 + 8));
-        const __half *h0 = reinterpret_cast<const __half *>(&s0);
-        const __half *h1 = reinterpret_cast<const __half *>(&s1);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            sk[j] = __half2float(h0[j]);
-            sk[8 + j] = __half2float(h1[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) bad |= !isfinite(sk[j]) || !(sk[j] > 0.0f);
-    }
+}  // namespace
 
-    // The raw binary16 rows stay in registers; the folded value w' = w * s_k
-    // (exact in float: 11 x 11 significant bits) is recomputed where needed.
-    uint4 raw[16];
-    float mx[8], mn[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        mx[c] = -INFINITY;
-        mn[c] = INFINITY;
-    }
-    if (active) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r)
-            raw[r] = __ldg(reinterpret_cast<const uint4 *>(W + (size_t)(k0 + r) * N + n));
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const __half *h = reinterpret_cast<const __half *>(&raw[r]);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float v = __fmul_rn(__half2float(h[c]), sk[r]);
-                bad |= !isfinite(v);
-                mx[c] = fmaxf(mx[c], v);
-                mn[c] = fminf(mn[c], v);
-            }
-        }
-    }
-    if (bad && active) report(status, AWQ_ERR_NONFINITE);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        red_max[warp][lane * 8 + c] = mx[c];
-        red_min[warp][lane * 8 + c] = mn[c];
+__global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __grid_constant__ CUtensorMap tmW,
+                                                                    const QuantParams p)
+{
+    extern __shared__ uint8_t qsmem_raw[];
+    QuantSmem &sm = *reinterpret_cast<QuantSmem *>(qsmem_raw + ((128u - (smem_u32(qsmem_raw) & 127u)) & 127u));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    if (tid == 0) {
+        prefetch_tmap(&tmW);
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        fence_barrier_init();
     }
     __syncthreads();
-    if (!active) return;
-
-    float sf[8], rsf[8];
-    int zc[8];
-    uint16_t sh[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        float a = red_max[0][lane * 8 + c], b = red_min[0][lane * 8 + c];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            a = fmaxf(a, red_max[i][lane * 8 + c]);
-            b = fminf(b, red_min[i][lane * 8 + c]);
-        }
-        float r = __fsub_rn(a, b);
-        if (r < 1e-5f) r = 1e-5f;
-        uint16_t bits = __half_as_ushort(__float2half_rn(__fdiv_rn(r, 15.0f)));
-        if ((bits & 0x7FFF) == 0) bits = 1;  // never a zero step
-        sh[c] = bits;
-        sf[c] = __half2float(__ushort_as_half(bits));
-        rsf[c] = __frcp_rn(sf[c]);
-        float zf = rintf(__fdiv_rn(-b, sf[c]));
-        zf = fminf(fmaxf(zf, 0.0f), 15.0f);
-        zc[c] = static_cast<int>(zf);
+    auto issue = [&](int t, int st) {
+        const int g = t / p.n_ctiles;
+        const int ct = t - g * p.n_ctiles;
+        mbar_arrive_expect_tx(&sm.full[st], kQTileBytes);
+        tma_load_2d(sm.stage[st], &tmW, &sm.full[st], ct * kQTileN, g * kGroup);
+    };
+    if (tid == 0) {
+        if (static_cast<int>(blockIdx.x) < p.tiles) issue(blockIdx.x, 0);
+        if (static_cast<int>(blockIdx.x + gridDim.x) < p.tiles) issue(blockIdx.x + gridDim.x, 1);
     }
 
-    uint32_t word[2][8];
+    bool ok = true, bad = false;
+    int it = 0;
+    for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++it) {
+        const int st = it & 1;
+        const int g = t / p.n_ctiles;
+        const int n0 = (t - g * p.n_ctiles) * kQTileN;
+        const int k0 = g * kGroup + 8 * warp;
+        // per-row channel scale: same for the whole warp (broadcast load)
+        const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(p.s + k0));
+        const uint16_t *sk = reinterpret_cast<const uint16_t *>(&sv);
+        if (ok && !mbar_wait(&sm.full[st], static_cast<uint32_t>(it >> 1) & 1u)) ok = false;
+
+        uint4 raw[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+        for (int j = 0; j < 8; ++j)
+            raw[j] = *reinterpret_cast<const uint4 *>(sm.stage[st] + ((8 * warp + j) * kQTileN + 8 * lane) * 2);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float sj = __half2float(__ushort_as_half(sk[j]));
+            bad |= !(sj > 0.0f) || !isfinite(sj);
+        }
+
+        // ---- pass 1: column max / min of w' over this thread's 8 rows
+        float mx[8], mn[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint32_t acc = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const __half *hr = reinterpret_cast<const __half *>(&raw[h * 8 + j]);
-                const float v = __fmul_rn(__half2float(hr[c]), sk[h * 8 + j]);
-                int q = rint_quotient(v, sf[c], rsf[c]) + zc[c];
-                q = min(max(q, 0), 15);
-                acc |= static_cast<uint32_t>(q) << (4 * j);
-            }
-            word[h][c] = acc;
+            mx[c] = -INFINITY;
+            mn[c] = INFINITY;
         }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        int32_t *dst = Q + (size_t)(k0 / 8 + h) * N + n;
-        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(word[h][0], word[h][1], word[h][2], word[h][3]);
-        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(word[h][4], word[h][5], word[h][6], word[h][7]);
-    }
-    if (warp == 0) {
-        uint4 sv;
-        sv.x = sh[0] | (static_cast<uint32_t>(sh[1]) << 16);
-        sv.y = sh[2] | (static_cast<uint32_t>(sh[3]) << 16);
-        sv.z = sh[4] | (static_cast<uint32_t>(sh[5]) << 16);
-        sv.w = sh[6] | (static_cast<uint32_t>(sh[7]) << 16);
-        *reinterpret_cast<uint4 *>(scales + (size_t)g * N + n) = sv;
-        uint32_t zw = 0;
+        for (int j = 0; j < 8; ++j) {
+            const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) zw |= static_cast<uint32_t>(zc[c]) << (4 * c);
-        zeros[(size_t)g * (N / 8) + n / 8] = static_cast<int32_t>(zw);
+            for (int c = 0; c < 8; ++c) {
+                const float v = fold(w[c], sk[j]);
+                mx[c] = fmax_nan(mx[c], v);
+                mn[c] = fmin_nan(mn[c], v);
+            }
+        }
+        *reinterpret_cast<float4 *>(&sm.red_max[warp][8 * lane]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+        *reinterpret_cast<float4 *>(&sm.red_max[warp][8 * lane + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
+        *reinterpret_cast<float4 *>(&sm.red_min[warp][8 * lane]) = make_float4(mn[0], mn[1], mn[2], mn[3]);
+        *reinterpret_cast<float4 *>(&sm.red_min[warp][8 * lane + 4]) = make_float4(mn[4], mn[5], mn[6], mn[7]);
+        __syncthreads();  // the stage is read, the partial extremes are written
+
+        // the stage is free: bring the tile two steps ahead
+        if (tid == 0 && t + 2 * static_cast<int>(gridDim.x) < p.tiles) issue(t + 2 * gridDim.x, st);
+
+        // ---- one thread per column: step, zero point, reciprocal, clamp flag
+        if (tid < kQTileN) {
+            float a = sm.red_max[0][tid], b = sm.red_min[0][tid];
+#pragma unroll
+            for (int i = 1; i < 16; ++i) {
+                a = fmax_nan(a, sm.red_max[i][tid]);
+                b = fmin_nan(b, sm.red_min[i][tid]);
+            }
+            const bool col_in = n0 + tid < p.N;
+            const bool fin = isfinite(a) && isfinite(b);
+            bad |= col_in && !fin;
+            if (!fin) {
+                a = 0.0f;
+                b = 0.0f;
+            }
+            float r = __fsub_rn(a, b);
+            if (r < 1e-5f) r = 1e-5f;
+            uint16_t bits = __half_as_ushort(__float2half_rn(__fdiv_rn(r, 15.0f)));
+            if ((bits & 0x7FFF) == 0) bits = 1;  // never a zero step
+            const float sf = __half2float(__ushort_as_half(bits));
+            float zf = rintf(__fdiv_rn(-b, sf));
+            zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+            const int z = static_cast<int>(zf);
+            // codes are monotone in w', so the extremes decide whether any clamps
+            const int qa = static_cast<int>(rintf(__fdiv_rn(a, sf))) + z;
+            const int qb = static_cast<int>(rintf(__fdiv_rn(b, sf))) + z;
+            sm.rsf[tid] = __frcp_rn(sf);
+            sm.cmag[tid] = kMagic + zf;
+            sm.step[tid] = sf;
+            sm.zc[tid] = z | ((qa > 15 || qb < 0) ? 0x100 : 0);
+            if (col_in) p.scales[static_cast<size_t>(g) * p.N + n0 + tid] = __ushort_as_half(bits);
+        }
+        __syncthreads();  // column parameters ready
+
+        if (tid < kQTileN / 8 && n0 + 8 * tid < p.N) {
+            uint32_t zw = 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) zw |= static_cast<uint32_t>(sm.zc[8 * tid + c] & 15) << (4 * c);
+            p.zeros[static_cast<size_t>(g) * (p.N / 8) + n0 / 8 + tid] = static_cast<int32_t>(zw);
+        }
+
+        // ---- pass 2: codes, packed 8 to a word (one word per column)
+        const int cb = 8 * lane;
+        int clamp_any = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) clamp_any |= sm.zc[cb + c] & 0x100;
+        uint32_t word[8];
+        if (!clamp_any) {
+#pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+                const int c0 = 2 * cp;
+                const unsigned long long rs2 = pk(sm.rsf[cb + c0], sm.rsf[cb + c0 + 1]);
+                const float m0 = sm.cmag[cb + c0], m1 = sm.cmag[cb + c0 + 1];
+                const unsigned long long cm2 = pk(m0, m1), ncm2 = pk(-m0, -m1);
+                uint32_t acc0 = 0u - kMagicWord, acc1 = 0u - kMagicWord;
+                float dmax0 = 0.0f, dmax1 = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
+                    const unsigned long long y2 = mul2(pk(fold(w[c0], sk[j]), fold(w[c0 + 1], sk[j])), rs2);
+                    const unsigned long long t2 = add2(y2, cm2);    // magic + z + rint(y)
+                    const unsigned long long r2 = add2(t2, ncm2);   // rint(y), exact
+                    float y0, y1, t0, t1, q0, q1;
+                    upk(y2, y0, y1);
+                    upk(t2, t0, t1);
+                    upk(r2, q0, q1);
+                    dmax0 = fmaxf(dmax0, fabsf(y0 - q0));
+                    dmax1 = fmaxf(dmax1, fabsf(y1 - q1));
+                    acc0 += __float_as_uint(t0) << (4 * j);
+                    acc1 += __float_as_uint(t1) << (4 * j);
+                }
+                word[c0] = acc0;
+                word[c0 + 1] = acc1;
+                // a code near a tie: redo the column's word with the IEEE quotient
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if ((h ? dmax1 : dmax0) >= kTieMargin) {
+                        const int c = c0 + h;
+                        const float sf = sm.step[cb + c];
+                        const int z = sm.zc[cb + c] & 15;
+                        uint32_t acc = 0;
+                        for (int j = 0; j < 8; ++j) {
+                            const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
+                            acc |= code_exact(fold(w[c], sk[j]), sf, z) << (4 * j);
+                        }
+                        word[c] = acc;
+                    }
+                }
+            }
+        } else {
+            // some column of this thread clamps: every code with the IEEE quotient
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float sf = sm.step[cb + c];
+                const int z = sm.zc[cb + c] & 15;
+                uint32_t acc = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
+                    acc |= code_exact(fold(w[c], sk[j]), sf, z) << (4 * j);
+                }
+                word[c] = acc;
+            }
+        }
+        if (n0 + cb < p.N) {
+            int32_t *dst = p.Q + static_cast<size_t>(g * 16 + warp) * p.N + n0 + cb;
+            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(word[0], word[1], word[2], word[3]);
+            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(word[4], word[5], word[6], word[7]);
+        }
     }
+    if (bad) report(p.status, AWQ_ERR_NONFINITE);
+    if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -298,11 +443,31 @@ cudaError_t launch_compute_scales(const float *m, int K, uint16_t *s, int32_t *s
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_pack(const __half *W, const __half *s, int K, int N, int32_t *Q,
-                                 __half *scales, int32_t *zeros, int32_t *status, cudaStream_t st)
+size_t quantize_smem_bytes() { return sizeof(QuantSmem) + 128; }
+
+cudaError_t configure_quantize()
 {
-    dim3 grid((N + 255) / 256, K / kGroup);
-    quantize_pack_kernel<<<grid, 256, 0, st>>>(W, s, K, N, Q, scales, zeros, status);
+    return cudaFuncSetAttribute(quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(quantize_smem_bytes()));
+}
+
+cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K, int N, int32_t *Q,
+                                 __half *scales, int32_t *zeros, int32_t *status, int num_sms,
+                                 cudaStream_t st)
+{
+    QuantParams prm{};
+    prm.s = s;
+    prm.Q = Q;
+    prm.scales = scales;
+    prm.zeros = zeros;
+    prm.status = status;
+    prm.K = K;
+    prm.N = N;
+    prm.G = K / kGroup;
+    prm.n_ctiles = (N + kQTileN - 1) / kQTileN;
+    prm.tiles = prm.G * prm.n_ctiles;
+    const int grid = prm.tiles < num_sms ? prm.tiles : num_sms;
+    quantize_pack_kernel<<<grid, kQThreads, quantize_smem_bytes(), st>>>(tmW, prm);
     return cudaGetLastError();
 }
 
