@@ -15,15 +15,17 @@
 namespace awq {
 
 // ------------------------------------------------------------------ act_stats
-// Block: 16 column chunks (8 channels each, one 16-byte load) x 16 row slices.
+// Block: 16 column chunks (8 channels each, one 16-byte load) x 64 row slices.
 // |x| is accumulated in double: every binary16 is a multiple of 2^-24 below
 // 2^16, so with R <= 8192 rows each partial and total sum is an exact double
-// and the order of the reduction cannot change the result.
-__global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict__ xcal, int R,
-                                                       int K, float *__restrict__ m,
-                                                       int32_t *status)
+// and the order of the reduction cannot change the result.  Each thread keeps
+// four rows' loads in flight.
+__global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restrict__ xcal, int R,
+                                                        int K, float *__restrict__ m,
+                                                        int32_t *status)
 {
-    __shared__ double part[16][129];
+    constexpr int kSlices = 64;
+    __shared__ double part[kSlices / 2][129];
     const int cc = threadIdx.x & 15;
     const int rs = threadIdx.x >> 4;
     const int k0 = blockIdx.x * 128 + cc * 8;
@@ -32,28 +34,41 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict
     for (int j = 0; j < 8; ++j) acc[j] = 0.0;
     bool bad = false;
     if (k0 < K) {
-        for (int r = rs; r < R; r += 16) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xcal + (size_t)r * K + k0));
-            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+        for (int r0 = rs; r0 < R; r0 += 4 * kSlices) {
+            uint4 v[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __half22float2(h[j]);
-                bad |= !isfinite(f.x) || !isfinite(f.y);
-                acc[2 * j] += fabs(static_cast<double>(f.x));
-                acc[2 * j + 1] += fabs(static_cast<double>(f.y));
+            for (int u = 0; u < 4; ++u) {
+                const int r = r0 + u * kSlices;
+                v[u] = r < R ? __ldg(reinterpret_cast<const uint4 *>(xcal + (size_t)r * K + k0))
+                             : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const __half2 *h = reinterpret_cast<const __half2 *>(&v[u]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __half22float2(h[j]);
+                    bad |= !isfinite(f.x) || !isfinite(f.y);
+                    acc[2 * j] += fabs(static_cast<double>(f.x));
+                    acc[2 * j + 1] += fabs(static_cast<double>(f.y));
+                }
             }
         }
     }
     if (bad) report(status, AWQ_ERR_NONFINITE);
+    // lanes l and l + 16 hold the same channels for two row slices
 #pragma unroll
-    for (int j = 0; j < 8; ++j) part[rs][cc * 8 + j] = acc[j];
+    for (int j = 0; j < 8; ++j) acc[j] += __shfl_down_sync(0xffffffffu, acc[j], 16);
+    if ((threadIdx.x & 16) == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[rs >> 1][cc * 8 + j] = acc[j];
+    }
     __syncthreads();
     if (threadIdx.x < 128) {
         const int k = blockIdx.x * 128 + threadIdx.x;
         if (k < K) {
             double s = 0.0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s += part[i][threadIdx.x];
+            for (int i = 0; i < kSlices / 2; ++i) s += part[i][threadIdx.x];
             m[k] = __double2float_rn(__ddiv_rn(s, static_cast<double>(R)));
         }
     }
@@ -81,16 +96,19 @@ __device__ __forceinline__ double scale_t(float mk)
     return __dsqrt_rn(fmax(static_cast<double>(mk), 1e-8));
 }
 
-// One block of 1024 threads: a min/max pass, then the rounding pass.
+// Every block first finds max m and min m over all K channels (plain float
+// compares: t = sqrt(max(m, 1e-8)) is monotone, so the largest and smallest t
+// are the square roots of the largest and smallest m, bit for bit), then
+// rounds its own 1024 channels.  No block depends on another.
 __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__restrict__ m, int K,
                                                              uint16_t *__restrict__ s,
                                                              int32_t *status)
 {
-    __shared__ double smax[32], smin[32];
+    __shared__ float smax[32], smin[32];
     __shared__ int sbad;
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
-    double tmax = 0.0, tmin = INFINITY;
+    float mx = 0.0f, mn = INFINITY;
     bool bad = false;
     for (int k = threadIdx.x; k < K; k += blockDim.x) {
         const float mk = m[k];
@@ -98,44 +116,43 @@ __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__res
             bad = true;
             continue;
         }
-        const double t = scale_t(mk);
-        tmax = fmax(tmax, t);
-        tmin = fmin(tmin, t);
+        mx = fmaxf(mx, mk);
+        mn = fminf(mn, mk);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        tmax = fmax(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-        tmin = fmin(tmin, __shfl_xor_sync(0xffffffffu, tmin, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) {
-        smax[warp] = tmax;
-        smin[warp] = tmin;
+        smax[warp] = mx;
+        smin[warp] = mn;
     }
     if (bad) atomicOr(&sbad, 1);
     __syncthreads();
     if (warp == 0) {
         const int nw = (blockDim.x + 31) >> 5;
-        tmax = lane < nw ? smax[lane] : 0.0;
-        tmin = lane < nw ? smin[lane] : INFINITY;
+        mx = lane < nw ? smax[lane] : 0.0f;
+        mn = lane < nw ? smin[lane] : INFINITY;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            tmax = fmax(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-            tmin = fmin(tmin, __shfl_xor_sync(0xffffffffu, tmin, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         }
         if (lane == 0) {
-            smax[0] = tmax;
-            smin[0] = tmin;
+            smax[0] = mx;
+            smin[0] = mn;
         }
     }
     __syncthreads();
     if (sbad) {
-        if (threadIdx.x == 0) report(status, AWQ_ERR_NONFINITE);
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(status, AWQ_ERR_NONFINITE);
         return;
     }
-    const double c = __dsqrt_rn(__dmul_rn(smax[0], smin[0]));
-    for (int k = threadIdx.x; k < K; k += blockDim.x)
-        s[k] = double_to_half_rn(__ddiv_rn(scale_t(m[k]), c));
+    const double c = __dsqrt_rn(__dmul_rn(scale_t(smax[0]), scale_t(smin[0])));
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k < K) s[k] = double_to_half_rn(__ddiv_rn(scale_t(m[k]), c));
 }
 
 // ------------------------------------------------------------------ quantize_pack
@@ -223,11 +240,30 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+// y - r for pairs, as fma(r, -1, y): exact when r = rint(y)
+__device__ __forceinline__ unsigned long long fms2(unsigned long long r, unsigned long long y)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(r), "l"(0xBF800000BF800000ull), "l"(y));
+    return d;
+}
 __device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b)
 {
     unsigned long long d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+
+// rint(fl(v / sf)) from y = v * fl(1 / sf), which lies within |y| * 2^-23 of
+// the exact quotient (|y| < 2^22 here: v and sf are finite, sf >= 2^-24);
+// only when y is within |y| * 2^-21 of a half-integer is the IEEE division
+// needed to decide.
+__device__ __forceinline__ float rint_quotient(float v, float sf, float rsf)
+{
+    const float y = __fmul_rn(v, rsf);
+    const float q = rintf(y);
+    if (fabsf(y - q) < 0.5f - fabsf(y) * 0x1p-21f) return q;
+    return rintf(__fdiv_rn(v, sf));
 }
 
 // The code decision with the correctly rounded quotient (the definition).
@@ -334,13 +370,14 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
             uint16_t bits = __half_as_ushort(__float2half_rn(__fdiv_rn(r, 15.0f)));
             if ((bits & 0x7FFF) == 0) bits = 1;  // never a zero step
             const float sf = __half2float(__ushort_as_half(bits));
-            float zf = rintf(__fdiv_rn(-b, sf));
+            const float rsf = __frcp_rn(sf);
+            float zf = rint_quotient(-b, sf, rsf);
             zf = fminf(fmaxf(zf, 0.0f), 15.0f);
             const int z = static_cast<int>(zf);
             // codes are monotone in w', so the extremes decide whether any clamps
-            const int qa = static_cast<int>(rintf(__fdiv_rn(a, sf))) + z;
-            const int qb = static_cast<int>(rintf(__fdiv_rn(b, sf))) + z;
-            sm.rsf[tid] = __frcp_rn(sf);
+            const int qa = static_cast<int>(rint_quotient(a, sf, rsf)) + z;
+            const int qb = static_cast<int>(rint_quotient(b, sf, rsf)) + z;
+            sm.rsf[tid] = rsf;
             sm.cmag[tid] = kMagic + zf;
             sm.step[tid] = sf;
             sm.zc[tid] = z | ((qa > 15 || qb < 0) ? 0x100 : 0);
@@ -374,14 +411,14 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
                 for (int j = 0; j < 8; ++j) {
                     const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
                     const unsigned long long y2 = mul2(pk(fold(w[c0], sk[j]), fold(w[c0 + 1], sk[j])), rs2);
-                    const unsigned long long t2 = add2(y2, cm2);    // magic + z + rint(y)
-                    const unsigned long long r2 = add2(t2, ncm2);   // rint(y), exact
-                    float y0, y1, t0, t1, q0, q1;
-                    upk(y2, y0, y1);
+                    const unsigned long long t2 = add2(y2, cm2);      // magic + z + rint(y)
+                    const unsigned long long r2 = add2(t2, ncm2);     // rint(y), exact
+                    const unsigned long long d2 = fms2(r2, y2);       // y - rint(y), exact
+                    float t0, t1, d0, d1;
                     upk(t2, t0, t1);
-                    upk(r2, q0, q1);
-                    dmax0 = fmaxf(dmax0, fabsf(y0 - q0));
-                    dmax1 = fmaxf(dmax1, fabsf(y1 - q1));
+                    upk(d2, d0, d1);
+                    dmax0 = fmaxf(dmax0, fabsf(d0));
+                    dmax1 = fmaxf(dmax1, fabsf(d1));
                     acc0 += __float_as_uint(t0) << (4 * j);
                     acc1 += __float_as_uint(t1) << (4 * j);
                 }
@@ -432,14 +469,14 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
 cudaError_t launch_act_stats(const __half *xcal, int R, int K, float *m, int32_t *status,
                              cudaStream_t st)
 {
-    act_stats_kernel<<<(K + 127) / 128, 256, 0, st>>>(xcal, R, K, m, status);
+    act_stats_kernel<<<(K + 127) / 128, 1024, 0, st>>>(xcal, R, K, m, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_compute_scales(const float *m, int K, uint16_t *s, int32_t *status,
                                   cudaStream_t st)
 {
-    compute_scales_kernel<<<1, 1024, 0, st>>>(m, K, s, status);
+    compute_scales_kernel<<<(K + 1023) / 1024, 1024, 0, st>>>(m, K, s, status);
     return cudaGetLastError();
 }
 
