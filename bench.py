@@ -214,7 +214,7 @@ def run_ours(args, rank, world, device):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic, "peak_source": peak_src,
-                "kernel": "small_m_kernel<1,prologue> (GEMV)",
+                "kernel": "gemv_kernel",
                 "bytes_per_launch_avg": round(alg_step / 4)}
 
     # ---- end to end through the public API: pinned host X in, host Y out, every step
