@@ -69,7 +69,8 @@ awq_status_t device_ready(int *sms)
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
             if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
-                awq::configure_gemv() != cudaSuccess || awq::configure_quantize() != cudaSuccess) {
+                awq::configure_gemv() != cudaSuccess || awq::configure_quantize() != cudaSuccess ||
+                awq::configure_tcs() != cudaSuccess) {
                 cudaGetLastError();
                 return AWQ_ERR_CUDA;
             }
@@ -146,6 +147,24 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;
         return from_cuda(awq::launch_gemv(gplan, tmQ, hX, hs, hsc, zeros, hY, m, k, n, dev_status, st));
+    }
+    // From about 40 tokens the small-batch layer needs more MMA rate than
+    // mma.sync gives: tcgen05 with the weights as the 128-row operand
+    // (measured on the 13B shapes: faster at 48 tokens, slower at 16 and 32).
+    int tcs_min_m = 40;
+#ifdef AWQ_TUNING
+    if (getenv("AWQ_TUNE_TCS_MINM")) tcs_min_m = atoi(getenv("AWQ_TUNE_TCS_MINM"));
+#endif
+    if (M >= tcs_min_m && M < 64) {
+        const awq::TcsPlan plan = awq::plan_tcs(m, k, n, sms);
+        if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
+                       static_cast<uint32_t>(plan.nt), CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 8,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+            return AWQ_ERR_CUDA;
+        e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
+        if (e != AWQ_OK) return e;
+        return from_cuda(awq::launch_tcs(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
     }
     if (M < 64) {
         const awq::SmallMPlan plan = awq::plan_small_m(m, k, n, sms);

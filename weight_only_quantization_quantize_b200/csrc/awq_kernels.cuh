@@ -62,6 +62,20 @@ cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensor
                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                       int32_t *status, cudaStream_t st);
 
+// matmul_tcs.cu -- 40 <= M < 64: tcgen05 with the weights as the 128-row operand
+struct TcsPlan {
+    int nt;        // tokens padded to a multiple of 16
+    int n_tiles;   // 128-column tiles
+    int splits;    // cluster size along K
+    int stage_bytes;
+    size_t smem;
+};
+TcsPlan plan_tcs(int M, int K, int N, int num_sms);
+cudaError_t configure_tcs();
+cudaError_t launch_tcs(const TcsPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
+                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                       int32_t *status, cudaStream_t st);
+
 // abi.cu -- host-side argument checks of the matmul (null, shape, alignment)
 awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                                 const uint16_t *scales, const int32_t *zeros, int64_t M,

@@ -1,0 +1,350 @@
+// matmul_tcs.cu -- Y = (X / s) . dequant(Q) for small batches (40 <= M < 64
+// tokens) on the 5th-generation tensor cores, with the roles of the operands
+// swapped: the dequantized weights are the 128-row A operand and the tokens
+// (padded to a multiple of 16) are the N dimension.
+//
+// Sources: lansai AWQ explainer (ai.lansai.wang/107648), "AWQ 的四步链路"
+// (Y = (X/s)(sW)); "Awq Quantization" (skillselion.com), "WQLinear Kernel
+// Variants" (GEMM kernel for batch sizes > 1), "Group Size Configuration",
+// "Zero-Point Quantization".
+//
+// At a few dozen tokens the layer does 2 M flops per weight: at HBM speed
+// that is more than the register-fed mma.sync path can issue on sm_100, while
+// tcgen05 has twice the rate and needs no register accumulators.
+//
+// One CTA = 128 output columns x one k range; the k ranges of a column tile are
+// the CTAs of a thread-block cluster (split-K, up to 8):
+//   warp 0      TMA ring (4 stages): X' tile [Nt tokens x 64 k] (128-byte
+//               swizzle; tokens beyond M read as zero), packed words
+//               [8 x 128]; cp.async of the group's steps and zero words.
+//   warp 1      allocates 64 TMEM columns; one lane issues
+//               tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = Nt, K = 16)
+//               x 4 per stage and commits each stage back to both rings.
+//   warps 2..9  dequantize: each writes (q - z) * step for 32 columns x 32 k
+//               as binary16 into the K-major, 128-byte-swizzled A operand
+//               (4-slot ring); then read the accumulator (tcgen05.ld) and push
+//               it to the cluster CTA that owns those columns (st.async); each
+//               CTA adds the k-split partials of its columns in rank order
+//               and writes Y.
+// Within each 8-channel chunk the contraction runs in the pair order
+// (0,4),(1,5),(2,6),(3,7) on both operands (X' is stored that way by the
+// pre-pass), which leaves the sum unchanged.
+#include "awq_kernels.cuh"
+
+namespace awq {
+
+namespace {
+
+constexpr int kBN = 128;               // output columns per CTA (MMA M)
+constexpr int kBK = 64;                // k per stage
+#ifndef TCS_LOAD_STAGES
+#define TCS_LOAD_STAGES 4
+#endif
+#ifndef TCS_A_STAGES
+#define TCS_A_STAGES 4
+#endif
+constexpr int kLoadStages = TCS_LOAD_STAGES;
+constexpr int kAStages = TCS_A_STAGES;  // dequantized A operand
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = 64 + 32 * kDequantWarps;
+constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 4 KB of packed words
+constexpr int kMetaBytes = 1024;              // 256 B steps + 64 B zero words, padded
+constexpr int kABytes = kBN * kBK * 2;        // 16 KB
+constexpr int kTmemCols = 64;
+
+struct Params {
+    const __half *scales;
+    const int32_t *zeros;
+    __half *Y;
+    int32_t *status;
+    int M, K, N;
+    int nt;           // tokens padded to a multiple of 16 (MMA N)
+    int splits;       // cluster size along K
+    int stage_bytes;  // X' tile + packed words + metadata
+    UnpackConsts uk;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tcs_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
+               const Params p)
+{
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *smem = align1024(smem_dyn);
+    uint8_t *aring = smem + kLoadStages * p.stage_bytes;  // 1 KB aligned
+    uint64_t *full_load = reinterpret_cast<uint64_t *>(aring + kAStages * kABytes);
+    uint64_t *empty_load = full_load + kLoadStages;
+    uint64_t *full_a = empty_load + kLoadStages;
+    uint64_t *empty_a = full_a + kAStages;
+    uint64_t *tmem_full = empty_a + kAStages;
+    uint64_t *recv_bar = tmem_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(recv_bar + 1);
+    // after the main loop the load ring is idle: it receives the pushed partials
+    float *recv = reinterpret_cast<float *>(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int split = blockIdx.x;  // == rank in the cluster
+    const int n0 = blockIdx.y * kBN;
+    const int KB = p.K / kBK;
+    const int kb_begin = static_cast<int>(static_cast<int64_t>(split) * KB / p.splits);
+    const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * KB / p.splits);
+    const int nkb = kb_end - kb_begin;
+    const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
+    const int xbytes = p.nt * 128;
+
+    pdl_launch_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kLoadStages; ++i) {
+            mbar_init(&full_load[i], 1 + 32);  // expect_tx + 32 cp.async arrivals
+            mbar_init(&empty_load[i], 1);      // MMA commit
+        }
+        for (int i = 0; i < kAStages; ++i) {
+            mbar_init(&full_a[i], kDequantWarps);
+            mbar_init(&empty_a[i], 1);         // MMA commit
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(recv_bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(p.splits * p.nt * cpo * 4));
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            prefetch_tmap(&tmQ);
+        }
+        pdl_wait();  // X' comes from the pre-pass kernel
+        for (int i = 0; i < nkb; ++i) {
+            const int kb = kb_begin + i;
+            const int st = i % kLoadStages;
+            if (i >= kLoadStages && !mbar_wait(&empty_load[st], ((i / kLoadStages) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t *stg = smem + st * p.stage_bytes;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full_load[st], static_cast<uint32_t>(xbytes + kQBytes));
+                tma_load_2d(stg, &tmX, &full_load[st], kb * kBK, 0);
+                tma_load_2d(stg + xbytes, &tmQ, &full_load[st], n0, kb * (kBK / 8));
+            }
+            uint8_t *meta = stg + xbytes + kQBytes;
+            const int g = (kb * kBK) / kGroup;
+            if (lane < 16) {
+                const int n = n0 + 8 * lane;
+                const bool in = n < p.N;
+                cp_async_16(meta + 16 * lane, p.scales + static_cast<size_t>(g) * p.N + (in ? n : 0),
+                            in ? 16u : 0u);
+            } else {
+                const int wi = n0 / 8 + (lane - 16);
+                const bool in = wi < p.N / 8;
+                cp_async_4(meta + 256 + 4 * (lane - 16),
+                           p.zeros + static_cast<size_t>(g) * (p.N / 8) + (in ? wi : 0), in ? 4u : 0u);
+            }
+            cp_async_arrive_noinc(&full_load[st]);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t idesc = tc_idesc_f16(kBN, p.nt);
+        for (int i = 0; i < nkb; ++i) {
+            const int st = i % kLoadStages;
+            const int as = i % kAStages;
+            if (!mbar_wait(&full_load[st], (i / kLoadStages) & 1) || !mbar_wait(&full_a[as], (i / kAStages) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t a0 = smem_u32(aring + as * kABytes);
+                const uint32_t b0 = smem_u32(smem + st * p.stage_bytes);
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    tc_mma(tmem_base, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                           (i > 0 || k > 0) ? 1u : 0u);
+                tc_commit(&empty_load[st]);
+                tc_commit(&empty_a[as]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            if (ok)
+                tc_commit(tmem_full);
+            else
+                report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ dequant
+        // warp d: column 32 * (d % 4) + lane, packed rows 4 * (d / 4) .. +3 of the stage
+        const int dw = warp - 2;
+        const int c = 32 * (dw & 3) + lane;
+        const int r0 = 4 * (dw >> 2);
+        const UnpackConsts uk = p.uk;
+        for (int i = 0; i < nkb; ++i) {
+            const int st = i % kLoadStages;
+            const int as = i % kAStages;
+            if (!mbar_wait(&full_load[st], (i / kLoadStages) & 1) ||
+                (i >= kAStages && !mbar_wait(&empty_a[as], ((i / kAStages) - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            const uint8_t *q = smem + st * p.stage_bytes + xbytes;
+            const uint8_t *meta = q + kQBytes;
+            const uint32_t abase = smem_u32(aring + as * kABytes);
+            const uint16_t sbits = reinterpret_cast<const uint16_t *>(meta)[c];
+            const uint32_t sc2 = static_cast<uint32_t>(sbits) | (static_cast<uint32_t>(sbits) << 16);
+            const uint32_t zw = reinterpret_cast<const uint32_t *>(meta + 256)[c >> 3];
+            uint32_t za, zb;
+            zero_constants((zw >> (4 * (c & 7))) & 15u, za, zb);
+            uint32_t w[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) w[r] = reinterpret_cast<const uint32_t *>(q + (r0 + r) * (kBN * 4))[c];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                uint32_t d[4];
+                unpack_minus_zero(w[r], za, zb, d, uk);
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[j]) : "r"(d[j]), "r"(sc2));
+                const uint32_t dst = abase + c * 128 + (((r0 + r) ^ (c & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
+                             "r"(o[2]), "r"(o[3])
+                             : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[as]);
+        }
+        if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    // Dequant warps read the accumulator: warp w reaches TMEM lanes
+    // 32 (w % 4) .. +31 (output columns) and takes half of the token columns.
+    // Every partial goes to the cluster rank owning its column: rank c / cpo,
+    // laid out there as [source rank][token][owned column].
+    const bool have_acc = warp >= 2 && ok && mbar_wait(tmem_full, 0);
+    if (warp >= 2 && !have_acc && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    // Every CTA of the cluster is past its main loop (its load ring, which
+    // receives the partials, is idle) and has initialized its barriers.
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (warp >= 2) {
+        tc_fence_after();
+        const int quarter = warp & 3;
+        const int col = quarter * 32 + lane;
+        const int half = (warp - 2) >> 2;
+        const int tb = half * (p.nt / 2);
+        const uint32_t owner = static_cast<uint32_t>(col / cpo);
+        const int lc = col - static_cast<int>(owner) * cpo;
+        const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
+        const uint32_t rbase = map_to_rank(smem_u32(recv), owner);
+        for (int t0 = tb; t0 < tb + p.nt / 2; t0 += 8) {
+            uint32_t v[8];
+            tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + t0, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float x = have_acc ? __uint_as_float(v[j]) : 0.0f;
+                const int off = ((split * p.nt + t0 + j) * cpo + lc) * 4;
+                st_async_f32(rbase + off, x, rbar);
+            }
+        }
+    }
+    cluster_arrive_release();  // pushes performed before the final wait completes anywhere
+    if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    for (int e = threadIdx.x; e < p.M * cpo; e += kThreads) {
+        const int tok = e / cpo;
+        const int lc = e - tok * cpo;
+        const int n = n0 + split * cpo + lc;
+        if (n >= p.N) continue;
+        float v = 0.0f;
+        for (int r = 0; r < p.splits; ++r) v += recv[(r * p.nt + tok) * cpo + lc];
+        p.Y[static_cast<size_t>(tok) * p.N + n] = __float2half_rn(v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+    cluster_wait_acquire();
+}
+
+}  // namespace
+
+TcsPlan plan_tcs(int M, int K, int N, int num_sms)
+{
+    TcsPlan pl{};
+    pl.nt = (M + 15) / 16 * 16;
+    pl.n_tiles = (N + kBN - 1) / kBN;
+    const int KB = K / kBK;
+    // Two CTAs per SM fit; the largest power-of-two split that keeps one wave
+    // and leaves every CTA at least four stages.
+    int splits = 1;
+    while (splits * 2 <= 8 && pl.n_tiles * splits * 2 <= 2 * num_sms && KB / (splits * 2) >= 4) splits *= 2;
+#ifdef AWQ_TUNING
+    if (const char *v = getenv("AWQ_TUNE_TCS_SPLITS")) {
+        int s = atoi(v);
+        while (s > 1 && (s & (s - 1))) --s;
+        if (s >= 1 && s <= 8 && KB / s >= 1) splits = s;
+    }
+#endif
+    pl.splits = splits;
+    pl.stage_bytes = pl.nt * 128 + kQBytes + kMetaBytes;
+    pl.smem = 1024 + static_cast<size_t>(kLoadStages) * pl.stage_bytes + static_cast<size_t>(kAStages) * kABytes +
+              256;
+    return pl;
+}
+
+cudaError_t configure_tcs()
+{
+    return cudaFuncSetAttribute(tcs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(plan_tcs(64, 128, 128, 1).smem));
+}
+
+cudaError_t launch_tcs(const TcsPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
+                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                       int32_t *status, cudaStream_t st)
+{
+    Params prm{scales, zeros, Y, status, M, K, N, plan.nt, plan.splits, plan.stage_bytes, unpack_consts()};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.splits, plan.n_tiles, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = plan.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, tcs_kernel, tmX, tmQ, prm);
+}
+
+}  // namespace awq
