@@ -15,6 +15,7 @@ Functions (names follow the C ABI):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -88,11 +89,18 @@ def status_string(code: int) -> str:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(t: torch.Tensor):
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _on(dev: torch.device):
+    """The device context for a call: a no-op when `dev` is already current."""
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
 
 
 def _need(t: torch.Tensor, dtype, ndim, name):
@@ -177,7 +185,7 @@ def w4a16_gemm(X, s, Q, scales, zeros, status=None, out=None, workspace=None) ->
     if wsz and workspace is None:
         workspace = torch.empty(wsz, dtype=torch.uint8, device=dev)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(dev):
+    with _on(dev):
         _check(lib().awq_w4a16_gemm(_ptr(X), _ptr(s), _ptr(Q), _ptr(scales), _ptr(zeros), M, K, N,
                                     _ptr(Y), _ptr(workspace), wbytes, _ptr(status), _stream(X)),
                "awq_w4a16_gemm")
@@ -195,7 +203,7 @@ def w4a16_gemv(X, s, Q, scales, zeros, status=None, out=None) -> torch.Tensor:
     N = Q.shape[1]
     dev = X.device
     Y = torch.empty(1, N, dtype=torch.float16, device=dev) if out is None else out
-    with torch.cuda.device(dev):
+    with _on(dev):
         _check(lib().awq_w4a16_gemv(_ptr(X), _ptr(s), _ptr(Q), _ptr(scales), _ptr(zeros), K, N,
                                     _ptr(Y), None, 0, _ptr(status), _stream(X)), "awq_w4a16_gemv")
     return Y
