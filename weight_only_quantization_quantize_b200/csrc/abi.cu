@@ -279,7 +279,7 @@ awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, 
     awq_status_t e = device_ready(&sms);
     if (e != AWQ_OK) return e;
     CUtensorMap tmW;
-    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, N, K, N * 2, 256, kGroup,
+    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W, N, K, N * 2, 128, kGroup,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return AWQ_ERR_CUDA;
     return from_cuda(awq::launch_quantize_pack(tmW, reinterpret_cast<const __half *>(s), static_cast<int>(K),

@@ -110,14 +110,25 @@ __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__res
     __syncthreads();
     float mx = 0.0f, mn = INFINITY;
     bool bad = false;
-    for (int k = threadIdx.x; k < K; k += blockDim.x) {
-        const float mk = m[k];
-        if (!isfinite(mk) || mk < 0.0f) {
-            bad = true;
-            continue;
+    // eight loads in flight per thread: the scan is bound by L2 latency otherwise
+    for (int k0 = threadIdx.x; k0 < K; k0 += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int k = k0 + u * blockDim.x;
+            v[u] = k < K ? m[k] : 0.0f;
         }
-        mx = fmaxf(mx, mk);
-        mn = fminf(mn, mk);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (k0 + u * blockDim.x >= K) continue;
+            const float mk = v[u];
+            if (!isfinite(mk) || mk < 0.0f) {
+                bad = true;
+                continue;
+            }
+            mx = fmaxf(mx, mk);
+            mn = fminf(mn, mk);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -156,32 +167,35 @@ __global__ void __launch_bounds__(1024) compute_scales_kernel(const float *__res
 }
 
 // ------------------------------------------------------------------ quantize_pack
-// Persistent CTAs (one per SM, 16 warps) walk tiles of one 128-row group x
-// 256 columns; TMA brings each 64 KB tile of W into a two-deep shared-memory
-// ring.  Warp w owns rows 8w..8w+7 (packed row w of the group) and lane l owns
-// columns 8l..8l+7, so every thread reads 8 x 16 bytes and writes one 32-byte
-// run of packed words.
+// Persistent CTAs (one per SM) of two independent halves of 8 warps.  Each half
+// walks its own tiles of one 128-row group x 128 columns, fed by its own TMA
+// double buffer of 32 KB tiles and synchronised by its own named barrier, so
+// one half's per-column phase overlaps the other half's streaming work.  In a
+// half, warp w owns rows 16w..16w+15 (packed rows 2w, 2w+1 of the group) and
+// lane l owns columns 4l..4l+3: every thread reads 16 x 8 bytes of the tile and
+// writes two 16-byte runs of packed words.
 //   pass 1  w' = w * s_k (exact: an fma of two binary16 into float), column
-//           max / min over the thread's 8 rows (NaN-propagating), then across
-//           the 16 warps in shared memory by one thread per column, which
+//           max / min over the thread's 16 rows (NaN-propagating), then across
+//           the half's 8 warps in shared memory by one thread per column, which
 //           also derives the column's step, zero point and reciprocal step.
 //   pass 2  the code decision rint(fl(w' / step)) without a division per
 //           weight: y = w' * fl(1 / step) lies within |y| * 2^-23 of the
 //           exact quotient, and adding 1.5 * 2^23 + z rounds y to an integer
-//           in the low mantissa bits (q = those bits, packed by one integer
-//           multiply-add per code).  A code whose y lies within 2^-18 of a
-//           half-integer is redone with the IEEE division, as is every code
-//           of a column whose extreme codes fall outside 0..15 (clamping).
+//           in the low mantissa bits (q = those bits, packed by one shift-add
+//           per code).  A code whose y lies within 2^-18 of a half-integer is
+//           redone with the IEEE division, as is every code of a column whose
+//           extreme codes fall outside 0..15 (clamping).
 // Pairs of columns go through the packed float32x2 multiply / add.
 namespace {
 
-constexpr int kQTileN = 256;                     // columns per tile
-constexpr int kQTileBytes = kGroup * kQTileN * 2;  // 64 KB of binary16
-constexpr int kQThreads = 512;                   // 16 warps: one packed row each
-constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+constexpr int kQTileN = 128;                       // columns per tile
+constexpr int kQTileBytes = kGroup * kQTileN * 2;  // 32 KB of binary16
+constexpr int kQHalfWarps = 8;
+constexpr int kQThreads = 2 * kQHalfWarps * 32;    // two halves of 8 warps
+constexpr float kMagic = 12582912.0f;              // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u;
 // sum_j kMagicBits * 16^j (mod 2^32): removed once from a word built with
-// one multiply-add per code from the raw bits of magic + code
+// one shift-add per code from the raw bits of magic + code
 constexpr uint32_t kMagicWord = kMagicBits * 0x11111111u;
 constexpr float kTieMargin = 0.5f - 0x1p-18f;
 
@@ -195,10 +209,10 @@ struct QuantParams {
     int tiles;
 };
 
-struct QuantSmem {
+struct alignas(128) QuantHalf {
     uint8_t stage[2][kQTileBytes];
-    float red_max[16][kQTileN];
-    float red_min[16][kQTileN];
+    float red_max[kQHalfWarps][kQTileN];
+    float red_min[kQHalfWarps][kQTileN];
     float rsf[kQTileN];   // fl(1 / step)
     float cmag[kQTileN];  // 1.5 * 2^23 + z
     float step[kQTileN];  // step as float (exact fallback)
@@ -279,10 +293,13 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
                                                                     const QuantParams p)
 {
     extern __shared__ uint8_t qsmem_raw[];
-    QuantSmem &sm = *reinterpret_cast<QuantSmem *>(qsmem_raw + ((128u - (smem_u32(qsmem_raw) & 127u)) & 127u));
-    const int tid = threadIdx.x;
+    QuantHalf *halves = reinterpret_cast<QuantHalf *>(qsmem_raw + ((128u - (smem_u32(qsmem_raw) & 127u)) & 127u));
+    const int half = threadIdx.x >> 8;
+    const int tid = threadIdx.x & 255;  // thread index within the half
     const int warp = tid >> 5;
     const int lane = tid & 31;
+    QuantHalf &sm = halves[half];
+    const uint32_t bar_id = 1 + half;
 
     if (tid == 0) {
         prefetch_tmap(&tmW);
@@ -291,6 +308,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
         fence_barrier_init();
     }
     __syncthreads();
+    // this half's tiles: first, then every (2 * gridDim.x)-th
+    const int t_first = 2 * blockIdx.x + half;
+    const int t_step = 2 * gridDim.x;
     auto issue = [&](int t, int st) {
         const int g = t / p.n_ctiles;
         const int ct = t - g * p.n_ctiles;
@@ -298,63 +318,64 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
         tma_load_2d(sm.stage[st], &tmW, &sm.full[st], ct * kQTileN, g * kGroup);
     };
     if (tid == 0) {
-        if (static_cast<int>(blockIdx.x) < p.tiles) issue(blockIdx.x, 0);
-        if (static_cast<int>(blockIdx.x + gridDim.x) < p.tiles) issue(blockIdx.x + gridDim.x, 1);
+        if (t_first < p.tiles) issue(t_first, 0);
+        if (t_first + t_step < p.tiles) issue(t_first + t_step, 1);
     }
 
     bool ok = true, bad = false;
     int it = 0;
-    for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++it) {
+    for (int t = t_first; t < p.tiles; t += t_step, ++it) {
         const int st = it & 1;
         const int g = t / p.n_ctiles;
         const int n0 = (t - g * p.n_ctiles) * kQTileN;
-        const int k0 = g * kGroup + 8 * warp;
-        // per-row channel scale: same for the whole warp (broadcast load)
-        const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(p.s + k0));
-        const uint16_t *sk = reinterpret_cast<const uint16_t *>(&sv);
+        const int k0 = g * kGroup + 16 * warp;
+        // per-row channel scales: the same for the whole warp (broadcast loads)
+        const uint4 sv0 = __ldg(reinterpret_cast<const uint4 *>(p.s + k0));
+        const uint4 sv1 = __ldg(reinterpret_cast<const uint4 *>(p.s + k0 + 8));
+        uint16_t sk[16];
+        *reinterpret_cast<uint4 *>(&sk[0]) = sv0;
+        *reinterpret_cast<uint4 *>(&sk[8]) = sv1;
         if (ok && !mbar_wait(&sm.full[st], static_cast<uint32_t>(it >> 1) & 1u)) ok = false;
 
-        uint4 raw[8];
+        uint2 raw[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            raw[j] = *reinterpret_cast<const uint4 *>(sm.stage[st] + ((8 * warp + j) * kQTileN + 8 * lane) * 2);
+        for (int j = 0; j < 16; ++j)
+            raw[j] = *reinterpret_cast<const uint2 *>(sm.stage[st] + ((16 * warp + j) * kQTileN + 4 * lane) * 2);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
             const float sj = __half2float(__ushort_as_half(sk[j]));
             bad |= !(sj > 0.0f) || !isfinite(sj);
         }
 
-        // ---- pass 1: column max / min of w' over this thread's 8 rows
-        float mx[8], mn[8];
+        // ---- pass 1: column max / min of w' over this thread's 16 rows
+        float mx[4], mn[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             mx[c] = -INFINITY;
             mn[c] = INFINITY;
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
             const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 const float v = fold(w[c], sk[j]);
                 mx[c] = fmax_nan(mx[c], v);
                 mn[c] = fmin_nan(mn[c], v);
             }
         }
-        *reinterpret_cast<float4 *>(&sm.red_max[warp][8 * lane]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
-        *reinterpret_cast<float4 *>(&sm.red_max[warp][8 * lane + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
-        *reinterpret_cast<float4 *>(&sm.red_min[warp][8 * lane]) = make_float4(mn[0], mn[1], mn[2], mn[3]);
-        *reinterpret_cast<float4 *>(&sm.red_min[warp][8 * lane + 4]) = make_float4(mn[4], mn[5], mn[6], mn[7]);
-        __syncthreads();  // the stage is read, the partial extremes are written
+        *reinterpret_cast<float4 *>(&sm.red_max[warp][4 * lane]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+        *reinterpret_cast<float4 *>(&sm.red_min[warp][4 * lane]) = make_float4(mn[0], mn[1], mn[2], mn[3]);
+        named_bar_sync(bar_id, 256);  // the stage is read, the partial extremes are written
 
-        // the stage is free: bring the tile two steps ahead
-        if (tid == 0 && t + 2 * static_cast<int>(gridDim.x) < p.tiles) issue(t + 2 * gridDim.x, st);
+        // the stage is free: bring this half's tile two steps ahead
+        if (tid == 0 && t + 2 * t_step < p.tiles) issue(t + 2 * t_step, st);
 
         // ---- one thread per column: step, zero point, reciprocal, clamp flag
         if (tid < kQTileN) {
             float a = sm.red_max[0][tid], b = sm.red_min[0][tid];
 #pragma unroll
-            for (int i = 1; i < 16; ++i) {
+            for (int i = 1; i < kQHalfWarps; ++i) {
                 a = fmax_nan(a, sm.red_max[i][tid]);
                 b = fmin_nan(b, sm.red_min[i][tid]);
             }
@@ -383,7 +404,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
             sm.zc[tid] = z | ((qa > 15 || qb < 0) ? 0x100 : 0);
             if (col_in) p.scales[static_cast<size_t>(g) * p.N + n0 + tid] = __ushort_as_half(bits);
         }
-        __syncthreads();  // column parameters ready
+        named_bar_sync(bar_id, 256);  // column parameters ready
 
         if (tid < kQTileN / 8 && n0 + 8 * tid < p.N) {
             uint32_t zw = 0;
@@ -392,73 +413,83 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
             p.zeros[static_cast<size_t>(g) * (p.N / 8) + n0 / 8 + tid] = static_cast<int32_t>(zw);
         }
 
-        // ---- pass 2: codes, packed 8 to a word (one word per column)
-        const int cb = 8 * lane;
+        // ---- pass 2: codes, packed 8 to a word: words[h][c] for packed row 2w + h
+        const int cb = 4 * lane;
         int clamp_any = 0;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) clamp_any |= sm.zc[cb + c] & 0x100;
-        uint32_t word[8];
+        for (int c = 0; c < 4; ++c) clamp_any |= sm.zc[cb + c] & 0x100;
+        uint32_t word[2][4];
         if (!clamp_any) {
 #pragma unroll
-            for (int cp = 0; cp < 4; ++cp) {
+            for (int cp = 0; cp < 2; ++cp) {
                 const int c0 = 2 * cp;
                 const unsigned long long rs2 = pk(sm.rsf[cb + c0], sm.rsf[cb + c0 + 1]);
                 const float m0 = sm.cmag[cb + c0], m1 = sm.cmag[cb + c0 + 1];
                 const unsigned long long cm2 = pk(m0, m1), ncm2 = pk(-m0, -m1);
-                uint32_t acc0 = 0u - kMagicWord, acc1 = 0u - kMagicWord;
-                float dmax0 = 0.0f, dmax1 = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
-                    const unsigned long long y2 = mul2(pk(fold(w[c0], sk[j]), fold(w[c0 + 1], sk[j])), rs2);
-                    const unsigned long long t2 = add2(y2, cm2);      // magic + z + rint(y)
-                    const unsigned long long r2 = add2(t2, ncm2);     // rint(y), exact
-                    const unsigned long long d2 = fms2(r2, y2);       // y - rint(y), exact
-                    float t0, t1, d0, d1;
-                    upk(t2, t0, t1);
-                    upk(d2, d0, d1);
-                    dmax0 = fmaxf(dmax0, fabsf(d0));
-                    dmax1 = fmaxf(dmax1, fabsf(d1));
-                    acc0 += __float_as_uint(t0) << (4 * j);
-                    acc1 += __float_as_uint(t1) << (4 * j);
-                }
-                word[c0] = acc0;
-                word[c0 + 1] = acc1;
-                // a code near a tie: redo the column's word with the IEEE quotient
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if ((h ? dmax1 : dmax0) >= kTieMargin) {
-                        const int c = c0 + h;
-                        const float sf = sm.step[cb + c];
-                        const int z = sm.zc[cb + c] & 15;
-                        uint32_t acc = 0;
-                        for (int j = 0; j < 8; ++j) {
-                            const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
-                            acc |= code_exact(fold(w[c], sk[j]), sf, z) << (4 * j);
+                    uint32_t acc0 = 0u - kMagicWord, acc1 = 0u - kMagicWord;
+                    float dmax0 = 0.0f, dmax1 = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int row = 8 * h + j;
+                        const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[row]);
+                        const unsigned long long y2 =
+                            mul2(pk(fold(w[c0], sk[row]), fold(w[c0 + 1], sk[row])), rs2);
+                        const unsigned long long t2 = add2(y2, cm2);   // magic + z + rint(y)
+                        const unsigned long long r2 = add2(t2, ncm2);  // rint(y), exact
+                        const unsigned long long d2 = fms2(r2, y2);    // y - rint(y), exact
+                        float t0, t1, d0, d1;
+                        upk(t2, t0, t1);
+                        upk(d2, d0, d1);
+                        dmax0 = fmaxf(dmax0, fabsf(d0));
+                        dmax1 = fmaxf(dmax1, fabsf(d1));
+                        acc0 += __float_as_uint(t0) << (4 * j);
+                        acc1 += __float_as_uint(t1) << (4 * j);
+                    }
+                    word[h][c0] = acc0;
+                    word[h][c0 + 1] = acc1;
+                    // a code near a tie: redo that word with the IEEE quotient
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if ((e ? dmax1 : dmax0) >= kTieMargin) {
+                            const int c = c0 + e;
+                            const float sf = sm.step[cb + c];
+                            const int z = sm.zc[cb + c] & 15;
+                            uint32_t acc = 0;
+                            for (int j = 0; j < 8; ++j) {
+                                const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[8 * h + j]);
+                                acc |= code_exact(fold(w[c], sk[8 * h + j]), sf, z) << (4 * j);
+                            }
+                            word[h][c] = acc;
                         }
-                        word[c] = acc;
                     }
                 }
             }
         } else {
             // some column of this thread clamps: every code with the IEEE quotient
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 const float sf = sm.step[cb + c];
                 const int z = sm.zc[cb + c] & 15;
-                uint32_t acc = 0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[j]);
-                    acc |= code_exact(fold(w[c], sk[j]), sf, z) << (4 * j);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint16_t *w = reinterpret_cast<const uint16_t *>(&raw[8 * h + j]);
+                        acc |= code_exact(fold(w[c], sk[8 * h + j]), sf, z) << (4 * j);
+                    }
+                    word[h][c] = acc;
                 }
-                word[c] = acc;
             }
         }
         if (n0 + cb < p.N) {
-            int32_t *dst = p.Q + static_cast<size_t>(g * 16 + warp) * p.N + n0 + cb;
-            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(word[0], word[1], word[2], word[3]);
-            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(word[4], word[5], word[6], word[7]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                int32_t *dst = p.Q + static_cast<size_t>(g * 16 + 2 * warp + h) * p.N + n0 + cb;
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(word[h][0], word[h][1], word[h][2], word[h][3]);
+            }
         }
     }
     if (bad) report(p.status, AWQ_ERR_NONFINITE);
@@ -480,7 +511,7 @@ cudaError_t launch_compute_scales(const float *m, int K, uint16_t *s, int32_t *s
     return cudaGetLastError();
 }
 
-size_t quantize_smem_bytes() { return sizeof(QuantSmem) + 128; }
+size_t quantize_smem_bytes() { return 2 * sizeof(QuantHalf) + 128; }
 
 cudaError_t configure_quantize()
 {
@@ -503,7 +534,8 @@ cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K,
     prm.G = K / kGroup;
     prm.n_ctiles = (N + kQTileN - 1) / kQTileN;
     prm.tiles = prm.G * prm.n_ctiles;
-    const int grid = prm.tiles < num_sms ? prm.tiles : num_sms;
+    const int pairs = (prm.tiles + 1) / 2;  // a CTA's two halves take two tiles at a time
+    const int grid = pairs < num_sms ? pairs : num_sms;
     quantize_pack_kernel<<<grid, kQThreads, quantize_smem_bytes(), st>>>(tmW, prm);
     return cudaGetLastError();
 }
