@@ -57,12 +57,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The files the decode GEMV kernel is compiled from: a stored ncu traffic figure
+# stays valid while none of them changes.
+GEMV_SOURCES = ("weight_only_quantization_quantize_b200/csrc/gemv.cu",
+                "weight_only_quantization_quantize_b200/csrc/awq_common.cuh",
+                "weight_only_quantization_quantize_b200/csrc/awq_kernels.cuh",
+                "include/awq_b200.h")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "weight_only_quantization_quantize_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+    for rel in GEMV_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(rel.encode() + f.read())
     return h.hexdigest()[:16]
 
 
