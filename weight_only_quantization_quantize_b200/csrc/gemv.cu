@@ -18,8 +18,7 @@
 // Structure (one CTA = 128 output columns x a k range; clusters split K):
 //   producer warp   TMA ring of 128-row groups (four 16 x 32-word boxes,
 //                   128-byte swizzle) + cp.async of the group's steps and zero
-//                   words; before the dependency wait it warms L2 with the
-//                   CTA's packed weights (programmatic dependent launch).
+//                   words; ring depth 8, 6 or 4 (see plan_gemv).
 //   4*KH consumers  32 columns per warp (KH warps split a group's rows); a
 //                   lane turns one 16-byte load (4 columns x 8 k) into four
 //                   even-form and four odd-form f16x2 operands with LOP3 only
@@ -371,6 +370,7 @@ cudaError_t configure_gemv_one()
 cudaError_t configure_gemv()
 {
     const cudaError_t r[] = {configure_gemv_one<8, 1>(), configure_gemv_one<8, 2>(),
+                             configure_gemv_one<6, 1>(), configure_gemv_one<6, 2>(),
                              configure_gemv_one<4, 1>(), configure_gemv_one<4, 2>()};
     for (cudaError_t x : r)
         if (x != cudaSuccess) return x;
@@ -395,14 +395,20 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     // splits is a power of two so each cluster rank owns 128 / splits columns.
     // Measured on the decode shapes (K 4096..14336, N 4096..28672): with at
     // most one 128-column tile per SM, an 8-deep ring and the largest split
-    // that still fits one wave at two CTAs per SM; with more tiles than SMs,
-    // a 4-deep ring and splits up to about six CTAs per SM for load balance.
+    // that still fits one wave at two CTAs per SM, or one split more with a
+    // 6-deep ring when that fits one wave at three CTAs per SM (the QKV shape:
+    // 5.8 us against 6.5); with more tiles than SMs, a 4-deep ring and splits
+    // up to about six CTAs per SM for load balance.
     int max_pow2 = 1;
     while (max_pow2 * 2 <= max_split) max_pow2 *= 2;
     int splits = 1;
     if (pl->n_tiles <= num_sms) {
         pl->stages = 8;
         while (splits * 2 <= max_pow2 && pl->n_tiles * splits * 2 <= 2 * num_sms) splits *= 2;
+        if (splits * 2 <= max_pow2 && pl->n_tiles * splits * 2 <= 3 * num_sms) {
+            splits *= 2;
+            pl->stages = 6;
+        }
     } else {
         pl->stages = 4;
         while (splits * 2 <= max_pow2 && pl->n_tiles * splits < 6 * num_sms) splits *= 2;
@@ -413,7 +419,10 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     if (splits < 1) splits = 1;
     while (splits & (splits - 1)) --splits;
     pl->kh = tune_env("AWQ_TUNE_KH", pl->kh);
-    pl->stages = tune_env("AWQ_TUNE_STAGES", pl->stages) <= 4 ? 4 : 8;
+    {
+        const int sv = tune_env("AWQ_TUNE_STAGES", pl->stages);
+        pl->stages = sv <= 4 ? 4 : (sv <= 6 ? 6 : 8);
+    }
 #endif
     // X' and the group sums live in shared memory: M * (groups per CTA) * 256 B
     // (+ 8 B per group half); find the smallest split at or above the choice that fits
@@ -454,6 +463,9 @@ cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __ha
     prm.mask_lo = 0x000F000Fu;
     prm.mask_hi = 0x00F000F0u;
     prm.magic = 0x64006400u;
+    if (plan.stages == 6)
+        return plan.kh == 2 ? launch_gemv_one<6, 2>(plan, tmQ, prm, st)
+                            : launch_gemv_one<6, 1>(plan, tmQ, prm, st);
     if (plan.stages == 4)
         return plan.kh == 2 ? launch_gemv_one<4, 2>(plan, tmQ, prm, st)
                             : launch_gemv_one<4, 1>(plan, tmQ, prm, st);
