@@ -106,18 +106,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
         : "memory");
 }
 
-// Hint the hardware to pull a 2-D tile into L2 (no shared-memory destination,
-// no completion to wait for).  Safe before griddepcontrol.wait: L2 is the
-// coherence point, so data a predecessor writes later is still seen by the
-// real loads issued after the wait.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-
 // ---------------------------------------------------------------- programmatic dependent launch
 // Allow the next kernel on the stream to start launching (its own prologue
 // then overlaps this kernel's tail).
@@ -157,16 +145,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
                  : "memory");
 }
 
-// ---------------------------------------------------------------- shared loads
-__device__ __forceinline__ uint4 lds128(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
-}
-
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
 {
@@ -179,13 +157,6 @@ __device__ __forceinline__ uint32_t cluster_ctarank()
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-                 "barrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
 }
 
 // Split cluster barrier: arrive (release) now, wait (acquire) later.
@@ -215,16 +186,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t ran
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
     return r;
-}
-
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
 }
 
 // ---------------------------------------------------------------- tensor cores (warp MMA)
