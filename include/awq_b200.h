@@ -153,6 +153,13 @@ AWQ_API awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int
  * (may be NULL when that size is 0); it holds X / s and is overwritten.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
  * (Y is then unspecified).
+ * Stream ordering: these kernels use programmatic dependent launch, so a call
+ * may start while the previous kernel on the stream is still finishing.  X is
+ * read only after that kernel has completed.  Q, scales and zeros are treated
+ * as layer state and may be read before it completes: they must not be
+ * written by a kernel that triggers programmatic dependent launch early.
+ * Ordinary kernels, copies and awq_quantize_pack complete before any
+ * dependent starts, so writing the weights with them is safe.
  */
 AWQ_API size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N);
 AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t *Q,

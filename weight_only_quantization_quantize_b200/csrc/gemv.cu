@@ -105,7 +105,9 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         mbar_arrive_expect_tx(recv_bar, KH * p.M * cpo * p.splits * 4);
     }
     __syncthreads();
-    cluster_arrive_release();  // barriers initialized; waited on before the first push
+    // Barriers initialized; waited on before the first push.  The init fence
+    // above already releases them to the cluster, so the arrival is relaxed.
+    cluster_arrive_relaxed();
 
     float acc[2][4];
 #pragma unroll
@@ -116,9 +118,15 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
         if (lane == 0) prefetch_tmap(&tmQ);
-        pdl_wait();
+        // The packed words, steps and zero words are layer state: no kernel that
+        // triggers its dependents early writes them (the quantization kernels
+        // run to completion first).  The first ring's worth is therefore issued
+        // before the wait on the previous kernel, so this call's weights stream
+        // while that kernel finishes.
+        const int pre = ng < S ? ng : S;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
+            if (it == pre) pdl_wait();
             const int st = it % S;
             if (it >= S && !mbar_wait(&empty[st], ((it / S) - 1) & 1)) {
                 ok = false;
@@ -146,6 +154,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
             }
             cp_async_arrive_noinc(&full[st]);
         }
+        pdl_wait();  // before this warp writes Y in the epilogue
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     } else {
         // ------------------------------------------------------------ consumers
@@ -158,41 +167,57 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
             const int sub = lane >> 4;              // two (token, group) pairs per warp pass
             const int c16 = lane & 15;
             const int pairs = p.M * ng;
-            for (int base = warp * 2; base < pairs; base += 2 * kConsumers) {
-                const int pair = base + sub;
-                const bool valid = pair < pairs;
-                const int tok = valid ? pair / ng : 0;
-                const int gl = valid ? pair - tok * ng : 0;
-                float e = 0.0f, o = 0.0f;
-                if (valid) {
-                    const int ch = gl * 16 + c16;
-                    const int k = (g_begin + gl) * kGroup + c16 * 8;
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(tok) * p.K + k));
-                    const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(p.s + k));
-                    const __half *xh = reinterpret_cast<const __half *>(&xv);
-                    const __half *sh = reinterpret_cast<const __half *>(&sv);
-                    __half q[8];
+            // Two passes' X and s loads are issued before either is used, so a CTA
+            // with up to 16 (token, group) pairs waits for one load latency.
+            constexpr int kBatch = 2;
+            for (int base = warp * 2; base < pairs; base += 2 * kConsumers * kBatch) {
+                uint4 xv[kBatch], sv[kBatch];
+                bool valid[kBatch];
+                int tok[kBatch], gl[kBatch];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        q[j] = __float2half_rn(__fdiv_rn(__half2float(xh[j]), __half2float(sh[j])));
-                    e = (__half2float(q[0]) + __half2float(q[2])) + (__half2float(q[4]) + __half2float(q[6]));
-                    o = (__half2float(q[1]) + __half2float(q[3])) + (__half2float(q[5]) + __half2float(q[7]));
-                    uint4 r;
-                    r.x = __half_as_ushort(q[0]) | (static_cast<uint32_t>(__half_as_ushort(q[4])) << 16);
-                    r.y = __half_as_ushort(q[2]) | (static_cast<uint32_t>(__half_as_ushort(q[6])) << 16);
-                    r.z = __half_as_ushort(q[1]) | (static_cast<uint32_t>(__half_as_ushort(q[5])) << 16);
-                    r.w = __half_as_ushort(q[3]) | (static_cast<uint32_t>(__half_as_ushort(q[7])) << 16);
-                    *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok) * chunks + (ch ^ (tok & 7))) * 16) = r;
+                for (int b = 0; b < kBatch; ++b) {
+                    const int pair = base + b * 2 * kConsumers + sub;
+                    valid[b] = pair < pairs;
+                    tok[b] = valid[b] ? pair / ng : 0;
+                    gl[b] = valid[b] ? pair - tok[b] * ng : 0;
+                    xv[b] = make_uint4(0u, 0u, 0u, 0u);
+                    sv[b] = xv[b];
+                    if (valid[b]) {
+                        const int k = (g_begin + gl[b]) * kGroup + c16 * 8;
+                        xv[b] = __ldg(reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(tok[b]) * p.K + k));
+                        sv[b] = __ldg(reinterpret_cast<const uint4 *>(p.s + k));
+                    }
                 }
-                // butterfly over the lanes of one group half (fixed order)
 #pragma unroll
-                for (int off = kLanesPerHalf / 2; off > 0; off >>= 1) {
-                    e += __shfl_xor_sync(0xffffffffu, e, off);
-                    o += __shfl_xor_sync(0xffffffffu, o, off);
+                for (int b = 0; b < kBatch; ++b) {
+                    float e = 0.0f, o = 0.0f;
+                    if (valid[b]) {
+                        const int ch = gl[b] * 16 + c16;
+                        const __half *xh = reinterpret_cast<const __half *>(&xv[b]);
+                        const __half *sh = reinterpret_cast<const __half *>(&sv[b]);
+                        __half q[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            q[j] = __float2half_rn(__fdiv_rn(__half2float(xh[j]), __half2float(sh[j])));
+                        e = (__half2float(q[0]) + __half2float(q[2])) + (__half2float(q[4]) + __half2float(q[6]));
+                        o = (__half2float(q[1]) + __half2float(q[3])) + (__half2float(q[5]) + __half2float(q[7]));
+                        uint4 r;
+                        r.x = __half_as_ushort(q[0]) | (static_cast<uint32_t>(__half_as_ushort(q[4])) << 16);
+                        r.y = __half_as_ushort(q[2]) | (static_cast<uint32_t>(__half_as_ushort(q[6])) << 16);
+                        r.z = __half_as_ushort(q[1]) | (static_cast<uint32_t>(__half_as_ushort(q[5])) << 16);
+                        r.w = __half_as_ushort(q[3]) | (static_cast<uint32_t>(__half_as_ushort(q[7])) << 16);
+                        *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok[b]) * chunks + (ch ^ (tok[b] & 7))) * 16) = r;
+                    }
+                    // butterfly over the lanes of one group half (fixed order)
+#pragma unroll
+                    for (int off = kLanesPerHalf / 2; off > 0; off >>= 1) {
+                        e += __shfl_xor_sync(0xffffffffu, e, off);
+                        o += __shfl_xor_sync(0xffffffffu, o, off);
+                    }
+                    if (valid[b] && (c16 % kLanesPerHalf) == 0)
+                        gmeta[(tok[b] * ng + gl[b]) * KH + c16 / kLanesPerHalf] =
+                            make_float2(fmaf(1024.0f, e, 64.0f * o), e + o);
                 }
-                if (valid && (c16 % kLanesPerHalf) == 0)
-                    gmeta[(tok * ng + gl) * KH + c16 / kLanesPerHalf] =
-                        make_float2(fmaf(1024.0f, e, 64.0f * o), e + o);
             }
             named_bar_sync(1, kCThreads);
         }
@@ -203,7 +228,9 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         const int khalf = warp >> 2;
         const int colw = 32 * slab + 4 * gq;
         const int tok0 = 2 * t;
-        const uint8_t *xbase = xpro;
+        // This lane's X' row (tokens beyond M never load it).  A chunk index
+        // it * 16 + r XOR-swizzled by gq < 8 equals it * 16 + (r ^ gq).
+        const uint8_t *xrow = xpro + static_cast<size_t>(gq) * chunks * 16;
         const uint32_t mlo = p.mask_lo, mhi = p.mask_hi, magic = p.magic;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
@@ -232,9 +259,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                 const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);
                 const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
                 uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-                if (gq < p.M)
-                    bx = *reinterpret_cast<const uint4 *>(
-                        xbase + (static_cast<size_t>(gq) * chunks + ((it * 16 + r) ^ gq)) * 16);
+                if (gq < p.M) bx = *reinterpret_cast<const uint4 *>(xrow + it * 256 + ((r ^ gq) << 4));
                 const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
                 uint32_t ev0[4], ev2[4], od1[4], od3[4];
 #pragma unroll
@@ -269,7 +294,8 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int c = 2 * tile + (i >> 1);
-                    const float z = static_cast<float>((zw >> (zsh + 4 * c)) & 15u);
+                    // the 4-bit zero as a float: 2^23 + z exactly, minus 2^23
+                    const float z = __int_as_float(((zw >> (zsh + 4 * c)) & 15u) | 0x4B000000u) - 8388608.0f;
                     const float2 gm = (i & 1) ? gm1 : gm0;
                     float pgrp = fmaf(R[tile][1][i], 0.0625f, R[tile][0][i]) - gm.x;
                     pgrp = fmaf(-z, gm.y, pgrp);
@@ -301,11 +327,12 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
             }
         }
     }
-    // Arrive (release: this thread's pushes are performed before it is seen);
-    // the matching wait is the last thing a CTA does, so no CTA exits while a
-    // push from or to it is still in flight, yet nobody idles on it: every CTA
-    // has pushed long before any finishes reducing.
-    cluster_arrive_release();
+    // Arrive once this thread's pushes are issued; the matching wait is the last
+    // thing a CTA does, so every CTA has issued its pushes before any exits.
+    // No release is needed: each owner waits on its own mbarrier for every
+    // byte pushed to it before it reduces, so no push into a CTA is in flight
+    // when that CTA leaves.  (A release here fenced on the pushes' completion.)
+    cluster_arrive_relaxed();
     // Reduce the columns this rank owns, partials summed in (rank, k-half) order.
     if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     const int lchunks = cpo / 8;

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(160, 1)
         mbar_arrive_expect_tx(recv_bar, p.M * cpo * p.splits * 4);
     }
     __syncthreads();
-    cluster_arrive_release();
+    cluster_arrive_relaxed();  // the init fence above releases the barriers
 
     float acc[2][MT][4];
 #pragma unroll
@@ -268,7 +268,9 @@ __global__ void __launch_bounds__(160, 1)
                 }
             }
     }
-    cluster_arrive_release();  // pushes performed before the final wait completes anywhere
+    // Arrive once the pushes are issued (no fence: every owner waits for all
+    // the bytes pushed to it before it reduces, hence before it exits).
+    cluster_arrive_relaxed();
     if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     const int lchunks = cpo / 8;
     for (int e = threadIdx.x; e < p.M * lchunks; e += kAllThreads) {

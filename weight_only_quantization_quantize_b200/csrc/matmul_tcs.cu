@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    cluster_arrive_release();  // pushes performed before the final wait completes anywhere
+    // Arrive once the pushes are issued (no fence: every owner waits for all
+    // the bytes pushed to it before it reduces, hence before it exits).
+    cluster_arrive_relaxed();
     if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     for (int e = threadIdx.x; e < p.M * cpo; e += kThreads) {
         const int tok = e / cpo;
