@@ -58,10 +58,12 @@ def configure(lib):
     lib.awq_oracle_act_stats.argtypes = [P, I64, I64, P]
     lib.awq_oracle_compute_scales.argtypes = [P, I64, P]
     lib.awq_oracle_quantize_pack.argtypes = [P, P, I64, I64, P, P, P]
+    lib.awq_oracle_quantize_pack_symmetric.argtypes = [P, P, I64, I64, P, P]
     lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
     lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
     for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
-              lib.awq_oracle_quantize_pack, lib.awq_oracle_dequant, lib.awq_oracle_matmul):
+              lib.awq_oracle_quantize_pack, lib.awq_oracle_quantize_pack_symmetric,
+              lib.awq_oracle_dequant, lib.awq_oracle_matmul):
         f.restype = ctypes.c_int
     return lib
 
@@ -133,13 +135,16 @@ def compute_scales(m) -> np.ndarray:
     return s.view(np.float16)
 
 
-def quantize_pack(W, s):
-    """Fold s into W, asymmetric 4-bit group-128 quantization, pack.
+def quantize_pack(W, s, zero_point: bool = True):
+    """Fold s into W, 4-bit group-128 quantization, pack.
 
     "Awq Quantization", "Group Size Configuration" / "Zero-Point
     Quantization"; lansai explainer, four-step chain ("真实量化/打包").
     W: binary16 [K, N] (Y = X W), s: binary16 [K].
-    Returns (Q int32 [K/8, N], scales float16 [K/128, N], zeros int32 [K/128, N/8]).
+    zero_point=True: asymmetric grid with a per-group zero point.
+    zero_point=False: symmetric grid (step from the largest magnitude, codes
+    stored with an implicit zero point of 8); zeros is then None.
+    Returns (Q int32 [K/8, N], scales float16 [K/128, N], zeros int32 [K/128, N/8] or None).
     """
     w = _h(W)
     sv = _h(s)
@@ -148,20 +153,34 @@ def quantize_pack(W, s):
         raise ValueError("s must have shape [K]")
     Q = np.zeros((max(K // 8, 1), N), dtype=np.int32)
     sc = np.zeros((max(K // GROUP, 1), N), dtype=np.uint16)
+    if not zero_point:
+        _check(_load().awq_oracle_quantize_pack_symmetric(_p(w), _p(sv), K, N, _p(Q), _p(sc)),
+               "quantize_pack_symmetric")
+        return Q, sc.view(np.float16), None
     z = np.zeros((max(K // GROUP, 1), max(N // 8, 1)), dtype=np.int32)
     _check(_load().awq_oracle_quantize_pack(_p(w), _p(sv), K, N, _p(Q), _p(sc), _p(z)),
            "quantize_pack")
     return Q, sc.view(np.float16), z
 
 
+def _zeros_ptr(zeros):
+    """(array, pointer) for a zeros tensor; None (symmetric weights) is NULL."""
+    if zeros is None:
+        return None, None
+    z = np.ascontiguousarray(zeros, dtype=np.int32)
+    return z, _p(z)
+
+
 def dequant(Q, scales, zeros) -> np.ndarray:
-    """w_hat = (q - z) * scale (the fake-quantized weights), float64 [K, N]."""
+    """w_hat = (q - z) * scale (the fake-quantized weights), float64 [K, N].
+
+    zeros=None: symmetric weights, z = 8 everywhere."""
     Q = np.ascontiguousarray(Q, dtype=np.int32)
     sc = _h(scales)
-    z = np.ascontiguousarray(zeros, dtype=np.int32)
+    z, zp = _zeros_ptr(zeros)
     K, N = Q.shape[0] * 8, Q.shape[1]
     out = np.empty((K, N), dtype=np.float64)
-    _check(_load().awq_oracle_dequant(_p(Q), _p(sc), _p(z), K, N, _p(out)), "dequant")
+    _check(_load().awq_oracle_dequant(_p(Q), _p(sc), zp, K, N, _p(out)), "dequant")
     return out
 
 
@@ -171,6 +190,7 @@ def matmul(X, s, Q, scales, zeros, cols=None, precision: int = 64, nthreads: int
     Lansai explainer, four-step chain: Y = (X/s)(sW).  precision=64 computes
     everything in double; precision=32 is the dequantise-then-float-matmul
     (IEEE float division for X/s, float accumulation, k ascending, no FMA).
+    zeros=None: symmetric weights (z = 8).
     X: binary16 [M, K].  Returns float64 [M, len(cols)].
     """
     x = _h(X)
@@ -179,14 +199,14 @@ def matmul(X, s, Q, scales, zeros, cols=None, precision: int = 64, nthreads: int
     sv = _h(s)
     Q = np.ascontiguousarray(Q, dtype=np.int32)
     sc = _h(scales)
-    z = np.ascontiguousarray(zeros, dtype=np.int32)
+    z, zp = _zeros_ptr(zeros)
     M, K = x.shape
     N = Q.shape[1]
     if cols is None:
         cols = np.arange(N, dtype=np.int64)
     cols = np.ascontiguousarray(cols, dtype=np.int64)
     Y = np.empty((M, cols.shape[0]), dtype=np.float64)
-    _check(_load().awq_oracle_matmul(_p(x), _p(sv), _p(Q), _p(sc), _p(z), M, K, N, _p(cols),
+    _check(_load().awq_oracle_matmul(_p(x), _p(sv), _p(Q), _p(sc), zp, M, K, N, _p(cols),
                                      cols.shape[0], _p(Y), int(precision), int(nthreads)),
            "matmul")
     return Y

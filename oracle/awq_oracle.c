@@ -23,6 +23,8 @@
  *        Quantization" (an offset handles asymmetric weight distributions).
  *   [P1] AWQ skill card on skillsmd.top, "quant_config" example
  *        (zero_point = True, q_group_size = 128, w_bit = 4).
+ *   [P3] also shows the flag zero_point = False ("symmetric quantization",
+ *        for symmetric weight distributions or kernels without zero points).
  *
  * Where the pages leave a step open, the reading taken is stated at the step
  * (marked READING).  Status codes mirror the CUDA library's numbering so the
@@ -222,23 +224,85 @@ int awq_oracle_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, in
 }
 
 /* ---------------------------------------------------------------------------
+ * Steps 3-6, symmetric variant -- [P3] "Zero-Point Quantization": with
+ * zero_point = False the 4-bit grid has no per-group offset.  The page gives
+ * only the flag.
+ * READINGS:
+ *   fold     w' = float(w) * float(s_k), as above
+ *   range    a = max(max |w'|, 1e-5f) over the group (exact)
+ *   step     scale_h = binary16_RNE(a / 7.0f), never 0: the grid is centred
+ *            at zero and the largest magnitude lands on level +-7
+ *   code     q = clamp(rint(w' / float(scale_h)), -8, 7) + 8, stored in the
+ *            same nibbles as the asymmetric codes (0..15); no zeros tensor
+ *   value    w_hat = (q - 8) * scale_h, i.e. the asymmetric decode with z = 8
+ * ------------------------------------------------------------------------ */
+int awq_oracle_quantize_pack_symmetric(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                                       int32_t *Q, uint16_t *scales)
+{
+    if (!W || !s || !Q || !scales)
+        return OR_ERR_NULL;
+    if (K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0)
+        return OR_ERR_SHAPE;
+    for (int64_t k = 0; k < K; ++k) {
+        float sk = h2f(s[k]);
+        if (!isfinite(sk) || !(sk > 0.0f))
+            return OR_ERR_NONFINITE;
+    }
+    for (int64_t i = 0; i < K * N; ++i)
+        if (!isfinite(h2f(W[i])))
+            return OR_ERR_NONFINITE;
+
+    int64_t G = K / GROUP;
+    memset(Q, 0, sizeof(int32_t) * (size_t)((K / 8) * N));
+    for (int64_t g = 0; g < G; ++g) {
+        for (int64_t n = 0; n < N; ++n) {
+            float amax = 0.0f;
+            for (int64_t k = g * GROUP; k < (g + 1) * GROUP; ++k) {
+                float w = h2f(W[k * N + n]) * h2f(s[k]);
+                if (fabsf(w) > amax) amax = fabsf(w);
+            }
+            if (amax < 1e-5f)
+                amax = 1e-5f;
+            uint16_t sh = f2h(amax / 7.0f);
+            if ((sh & 0x7fff) == 0)
+                sh = 1;
+            float sf = h2f(sh);
+            scales[g * N + n] = sh;
+            for (int64_t k = g * GROUP; k < (g + 1) * GROUP; ++k) {
+                float w = h2f(W[k * N + n]) * h2f(s[k]);
+                float level = nearbyintf(w / sf);   /* half-to-even */
+                if (level < -8.0f) level = -8.0f;
+                if (level > 7.0f) level = 7.0f;
+                int32_t q = (int32_t)level + 8;
+                Q[(k / 8) * N + n] |= (int32_t)((uint32_t)q << (4 * (k % 8)));
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* ---------------------------------------------------------------------------
  * Step 7 -- dequantization (the pages' "伪量化" fake quantization: simulate the
  * low-bit weights in floating point).  w_hat[k,n] = (q - z) * scale_h, which
- * is exact in double.  Output [K, N] row-major.
+ * is exact in double; zeros == NULL means the symmetric grid (z = 8).  Output
+ * [K, N] row-major.
  * ------------------------------------------------------------------------ */
 static int code_at(const int32_t *Q, int64_t N, int64_t k, int64_t n)
 {
     return (int)(((uint32_t)Q[(k / 8) * N + n] >> (4 * (k % 8))) & 0xf);
 }
+/* zeros == NULL: symmetric weights, every zero point is 8 */
 static int zero_at(const int32_t *zeros, int64_t N, int64_t g, int64_t n)
 {
+    if (!zeros)
+        return 8;
     return (int)(((uint32_t)zeros[g * (N / 8) + n / 8] >> (4 * (n % 8))) & 0xf);
 }
 
 int awq_oracle_dequant(const int32_t *Q, const uint16_t *scales, const int32_t *zeros,
                        int64_t K, int64_t N, double *What)
 {
-    if (!Q || !scales || !zeros || !What)
+    if (!Q || !scales || !What)
         return OR_ERR_NULL;
     if (K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0)
         return OR_ERR_SHAPE;
@@ -315,7 +379,7 @@ int awq_oracle_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                       int64_t N, const int64_t *cols, int64_t ncols, double *Y,
                       int precision, int nthreads)
 {
-    if (!X || !s || !Q || !scales || !zeros || !cols || !Y)
+    if (!X || !s || !Q || !scales || !cols || !Y)   /* zeros may be NULL (symmetric) */
         return OR_ERR_NULL;
     if (M < 1 || K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0 || ncols < 1)
         return OR_ERR_SHAPE;

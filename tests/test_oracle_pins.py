@@ -407,3 +407,107 @@ def test_activation_aware_scaling_beats_plain_rtn_on_outlier_data():
     ea = np.linalg.norm(ya - ref)
     er = np.linalg.norm(yr - ref)
     assert ea < er, (ea, er)
+
+
+# --------------------------------------------------------------------------
+# symmetric variant ("Zero-Point Quantization": zero_point False)
+# --------------------------------------------------------------------------
+def test_symmetric_hand_worked_group(golden_dir):
+    fx = json.load(open(os.path.join(golden_dir, "hand_group_symmetric_k128_n8.json")))
+    W = _golden_W(fx)
+    s = np.ones(fx["K"], dtype=np.float16)
+    Q, sc, z = oracle.quantize_pack(W, s, zero_point=False)
+    assert z is None
+    exp = fx["expected"]
+    assert [f"{v:#06x}" for v in sc.view(np.uint16)[0]] == [e.lower() for e in exp["scales_bits"]]
+    assert [(int(Q[0, 0]) >> (4 * j)) & 15 for j in range(8)] == exp["codes_col0_rows0to7"]
+    qh = exp["Q_hex_by_column"]
+    for c in range(8):
+        spec = qh[f"col{c}"]
+        for r in range(16):
+            if "all" in spec:
+                want = spec["all"]
+            elif "row0" in spec:
+                want = spec["row0"] if r == 0 else spec["rows1to15"]
+            else:
+                want = spec["even_rows"] if r % 2 == 0 else spec["odd_rows"]
+            assert Q[r, c] == _hex32(want), (c, r)
+    wh = oracle.dequant(Q, sc, None)
+    assert wh[:9, 0].tolist() == exp["dequant_col0_rows0to8"]
+
+
+def _textbook_symmetric_rtn(W16):
+    """Plain symmetric round-to-nearest, 4 bits (levels -8..7), groups of 128 rows.
+
+    Vectorised numpy float32, written independently of the oracle's loops.
+    Returns codes (level + 8) [K, N] and scales (float16) [G, N].
+    """
+    K, N = W16.shape
+    w = W16.astype(np.float32).reshape(K // 128, 128, N)
+    a = np.maximum(np.abs(w).max(axis=1), np.float32(1e-5))
+    scale = (a / np.float32(7)).astype(np.float16)
+    scale[scale == 0] = np.float16(2.0 ** -24)
+    level = np.clip(np.rint(w / scale.astype(np.float32)[:, None, :]), -8, 7)
+    return (level + 8).reshape(K, N).astype(np.int64), scale
+
+
+@pytest.mark.parametrize("K,N,sigma", [(128, 8, 0.02), (512, 264, 0.02), (384, 40, 3.0)])
+def test_symmetric_equals_textbook_rtn_when_s_is_one(K, N, sigma):
+    rng = np.random.default_rng(K * 3 + N)
+    W = (rng.standard_normal((K, N)) * sigma).astype(np.float16)
+    Q, sc, _ = oracle.quantize_pack(W, np.ones(K, np.float16), zero_point=False)
+    codes, _ = _unpack(Q, np.zeros((K // 128, N // 8), np.int32), K, N)
+    q_ref, s_ref = _textbook_symmetric_rtn(W)
+    assert np.array_equal(sc.view(np.uint16), s_ref.view(np.uint16))
+    assert np.array_equal(codes, q_ref)
+
+
+def test_symmetric_negation_bounds_and_implicit_zero_point():
+    L = synth.make_layer(1, 0, M=1, K=1024, N=512, R=128)
+    s = oracle.compute_scales(oracle.act_stats(L.Xcal.numpy()))
+    W = L.W.numpy()
+    K, N = W.shape
+    Q, sc, _ = oracle.quantize_pack(W, s, zero_point=False)
+    codes, _ = _unpack(Q, np.zeros((K // 128, N // 8), np.int32), K, N)
+    # every |w'| <= max |w'| = 7 steps (up to the step's binary16 rounding): no
+    # level -8, nothing clamps, and rint is odd-symmetric under half-to-even
+    assert codes.min() >= 1 and codes.max() <= 15
+    Qn, scn, _ = oracle.quantize_pack(-W, s, zero_point=False)
+    cn, _ = _unpack(Qn, np.zeros((K // 128, N // 8), np.int32), K, N)
+    assert np.array_equal(scn.view(np.uint16), sc.view(np.uint16))
+    assert np.array_equal(cn, 16 - codes)
+    # round trip within half a step; the largest magnitude of a group lands on +-7
+    wf = (W.astype(np.float32) * s.astype(np.float32)[:, None]).astype(np.float64)
+    wg = wf.reshape(K // 128, 128, N)
+    sfg = sc.astype(np.float64)[:, None, :]
+    wh = (codes.reshape(K // 128, 128, N) - 8) * sfg
+    assert np.all(np.abs(wg - wh) <= 0.5 * sfg * (1 + 2.0 ** -9))
+    am = np.abs(wg).argmax(axis=1)
+    lv = np.take_along_axis(codes.reshape(K // 128, 128, N), am[:, None, :], axis=1)[:, 0, :] - 8
+    assert np.all(np.abs(lv) == 7)
+    # no zeros tensor means a zero point of 8 everywhere
+    eights = np.full((K // 128, N // 8), np.int32(np.int64(0x88888888).astype(np.uint32).astype(np.int32)))
+    assert np.array_equal(oracle.dequant(Q, sc, None), oracle.dequant(Q, sc, eights))
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 128, 8), (4, 512, 40)])
+def test_symmetric_matmul_lossless_grid_equals_plain_xw(M, K, N):
+    # folded weights on each group's symmetric grid (levels -7..7, both ends
+    # present): quantization is lossless and Y must equal X W exactly
+    rng = np.random.default_rng(M + K + N)
+    G = K // 128
+    step = 2.0 ** rng.integers(-9, -4, (G, N))
+    level = rng.integers(-7, 8, (K, N))
+    level[0::128, :] = -7
+    level[1::128, :] = 7
+    s = 2.0 ** rng.integers(-2, 3, K)
+    W = (level * np.repeat(step, 128, axis=0)) / s[:, None]
+    Wh = W.astype(np.float16)
+    assert np.array_equal(Wh.astype(np.float64), W)
+    Q, sc, z = oracle.quantize_pack(Wh, s.astype(np.float16), zero_point=False)
+    codes, _ = _unpack(Q, np.zeros((G, N // 8), np.int32), K, N)
+    assert np.array_equal(codes, level + 8)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    Y = oracle.matmul(X, s.astype(np.float16), Q, sc, None, precision=64)
+    ref = X.astype(np.float64) @ W
+    assert np.max(np.abs(Y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
