@@ -135,8 +135,10 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def build_layers(awq, nlayers, device, workload=WORKLOAD_ID):
-    """Quantize `nlayers` distinct synthetic layers on the GPU (kept packed)."""
+def build_layers(awq, nlayers, device, workload=WORKLOAD_ID, zero_point=True):
+    """Quantize `nlayers` distinct synthetic layers on the GPU (kept packed).
+
+    zero_point=False: symmetric weights (no zeros tensor; p["z"] is None)."""
     wl = synth.WORKLOADS[workload]
     layers = []
     for li in range(nlayers):
@@ -144,7 +146,7 @@ def build_layers(awq, nlayers, device, workload=WORKLOAD_ID):
         for si, (K, N, label) in enumerate(wl.shapes):
             L = synth.make_layer(workload, li, M=1, K=K, N=N, R=wl.R, device=device, shape_id=si)
             s = awq.compute_scales(awq.act_stats(L.Xcal))
-            Q, sc, z = awq.quantize_pack(L.W, s)
+            Q, sc, z = awq.quantize_pack(L.W, s, zero_point=zero_point)
             projs.append(dict(K=K, N=N, label=label, X=L.X, s=s, Q=Q, sc=sc, z=z,
                               Y=torch.empty(1, N, dtype=torch.float16, device=device)))
             del L
@@ -243,6 +245,8 @@ def run_ours(args, rank, world, device):
         extra["prefill_7b_m4096"] = run_prefill(awq, device, peaks)
         extra["quantize_7b_layer"] = run_quantize(awq, device, layers, peaks)
         extra["small_batch_13b_m48"] = run_small_batch(awq, device, peaks)
+        extra["quantize_7b_layer_symmetric"] = run_quantize(awq, device, layers, peaks, zero_point=False)
+        extra["decode_7b_symmetric"] = run_decode_symmetric(awq, device, peaks, nlayers)
 
     cpu = run_cpu_baseline(rank, world) if rank == 0 else None
     return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, launches=launches,
@@ -375,8 +379,45 @@ def run_small_batch(awq, device, peaks, M=48, reps=10):
             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "includes": "X/s pre-pass + 4 GEMMs"}
 
 
-def run_quantize(awq, device, layers, peaks, reps=5):
-    """act_stats + compute_scales + quantize_pack over one 7B layer (fp16 W read once)."""
+def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5):
+    """The decode step on symmetric weights (zeros = NULL), timed like the headline.
+
+    Algorithmic bytes: 0.5 B per weight + 2 B per 128 weights (no zero points)."""
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    layers = build_layers(awq, nlayers, device, zero_point=False)
+
+    def step(i):
+        for p in layers[i % nlayers]:
+            awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], None, out=p["Y"])
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g, layers
+    wbytes = sum(K * N * (0.5 + 2 / 128) for K, N, _ in wl.shapes)
+    gbs = wbytes * steps / (ms * 1e-3) / 1e9
+    return {"ms_per_step": round(ms / steps, 5), "weight_gbs": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "bytes": "0.5 B/weight codes + fp16 step per 128 weights; no zero points",
+            "l2": f"{nlayers} distinct layers rotated", "timing": "CUDA graph, CUDA events"}
+
+
+def run_quantize(awq, device, layers, peaks, reps=5, zero_point=True):
+    """act_stats + compute_scales + quantize_pack over one 7B layer (fp16 W read once).
+
+    zero_point=False times the symmetric quantizer (no zero points written)."""
     wl = synth.WORKLOADS[WORKLOAD_ID]
     ins = []
     for si, (K, N, label) in enumerate(wl.shapes):
@@ -390,13 +431,14 @@ def run_quantize(awq, device, layers, peaks, reps=5):
         e0.record()
         for L in ins:
             s = awq.compute_scales(awq.act_stats(L.Xcal))
-            awq.quantize_pack(L.W, s)
+            awq.quantize_pack(L.W, s, zero_point=zero_point)
         e1.record()
         torch.cuda.synchronize()
         if r >= 2:
             times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
-    moved = sum(2 * L.K * L.N + weight_bytes(L.K, L.N) + 2 * L.R * L.K for L in ins)
+    packed = weight_bytes if zero_point else (lambda K, N: K * N * (0.5 + 2 / 128))
+    moved = sum(2 * L.K * L.N + packed(L.K, L.N) + 2 * L.R * L.K for L in ins)
     gbs = moved / (ms * 1e-3) / 1e9
     return {"ms_per_layer": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
             "bytes": "fp16 W read + packed write + calibration rows"}

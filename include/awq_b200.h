@@ -38,7 +38,8 @@
  *                               of row 8*k8 + j, column n (sequential nibbles)
  *   scales  binary16 [G, N]     per-group step of the 4-bit grid
  *   zeros   int32 [G, N/8]      bits [4j, 4j+4) of zeros[g, n8] hold the zero
- *                               point of column 8*n8 + j
+ *                               point of column 8*n8 + j; absent (NULL) for
+ *                               symmetric weights, whose zero point is 8
  *   X       binary16 [M, K]     activations;  Y binary16 [M, N]
  */
 #ifndef AWQ_B200_H
@@ -63,7 +64,7 @@ extern "C" {
 #define AWQ_MAX_K 262144
 #define AWQ_MAX_N 1048576
 #define AWQ_MAX_M 1048576
-#define AWQ_ABI_VERSION 1
+#define AWQ_ABI_VERSION 2  /* 2: symmetric weights (quantize + NULL zeros) */
 
 typedef enum {
     AWQ_OK = 0,
@@ -134,6 +135,23 @@ AWQ_API awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int
                                int32_t *dev_status, awq_stream_t stream);
 
 /*
+ * Symmetric variant -- "Awq Quantization", "Zero-Point Quantization"
+ * (zero_point False: no per-group offset, for symmetric weight distributions
+ * and for kernels without zero points).  The page names only the flag; this
+ * library reads it as a grid centred at zero whose largest level is 7 steps:
+ *   a       = max(max |w'|, 1e-5f)
+ *   scale_h = binary16_RNE(a / 7)  (the smallest subnormal if that is 0)
+ *   q       = clamp(rint(w' / scale_h), -8, 7) + 8          (rint: ties to even)
+ * i.e. the asymmetric codes with z = 8.  No zeros tensor is written; pass
+ * zeros = NULL to the matmul entry points for these weights.
+ *   W, s, K, N, Q, scales as for awq_quantize_pack.
+ * Device errors: as for awq_quantize_pack.
+ */
+AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16_t *s, int64_t K,
+                                         int64_t N, int32_t *Q, uint16_t *scales,
+                                         int32_t *dev_status, awq_stream_t stream);
+
+/*
  * Fused-dequantization matmul -- lansai explainer, "AWQ 的四步链路"
  * (Y = (X/s)(sW)); "Awq Quantization", "WQLinear Kernel Variants" (GEMV for
  * batch size 1, GEMM for batches).
@@ -148,7 +166,8 @@ AWQ_API awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int
  *   X binary16 [1, K], Y binary16 [1, N].
  * awq_w4a16_gemm takes any 1 <= M <= AWQ_MAX_M and picks its tile path
  * internally (register-fed tensor cores for M < 64, tcgen05/TMEM for M >= 64).
- *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack.
+ *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack;
+ *   zeros = NULL for weights from awq_quantize_pack_symmetric (zero point 8).
  * Workspace: caller-owned device memory of at least *_workspace_size() bytes
  * (may be NULL when that size is 0); it holds X / s and is overwritten.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out

@@ -52,7 +52,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.awq_abi_version() == 1
+    assert L.awq_abi_version() == 2
     for code, name in awq.STATUS.items():
         assert awq.status_string(code).startswith(name)
     assert awq.status_string(99) == "AWQ_ERR_UNKNOWN"
@@ -72,7 +72,10 @@ def gemm(L, X=A, s=A, Q=A, sc=A, z=A, M=64, K=4096, N=4096, Y=A, ws=A, wsb=1 << 
 
 def test_matmul_validation(L):
     assert gemm(L, X=0) == awq.ERR_NULL
-    assert gemm(L, z=0) == awq.ERR_NULL
+    # zeros = NULL is legal (symmetric weights); the other checks still apply
+    assert gemm(L, z=0, K=100) == awq.ERR_SHAPE
+    assert gemm(L, z=0, Y=0) == awq.ERR_NULL
+    assert gemm(L, z=MIS) == awq.ERR_ALIGN
     assert gemm(L, Y=0) == awq.ERR_NULL
     assert gemm(L, K=100) == awq.ERR_SHAPE            # K % 128
     assert gemm(L, K=0) == awq.ERR_SHAPE
@@ -97,6 +100,14 @@ def test_quantize_and_stats_validation(L):
     assert q(P(A), P(A), 192, 8, P(A), P(A), P(A), None, None) == awq.ERR_SHAPE
     assert q(P(A), P(A), 128, 4, P(A), P(A), P(A), None, None) == awq.ERR_SHAPE
     assert q(P(A), P(MIS), 128, 8, P(A), P(A), P(A), None, None) == awq.ERR_ALIGN
+    assert q(P(A), P(A), 128, 8, P(A), P(A), P(0), None, None) == awq.ERR_NULL   # zeros required
+    qs = L.awq_quantize_pack_symmetric
+    assert qs(P(0), P(A), 128, 8, P(A), P(A), None, None) == awq.ERR_NULL
+    assert qs(P(A), P(A), 128, 8, P(A), P(0), None, None) == awq.ERR_NULL
+    assert qs(P(A), P(A), 192, 8, P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert qs(P(A), P(A), 128, 12, P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert qs(P(A), P(A), 128, 8, P(MIS), P(A), None, None) == awq.ERR_ALIGN
+    assert qs(P(A), P(A), 128, 8, P(A), P(A), P(A + 1), None) == awq.ERR_ALIGN
     st = L.awq_act_stats
     assert st(P(A), 0, 1024, P(A), None, None) == awq.ERR_SHAPE       # empty calibration
     assert st(P(A), 8193, 1024, P(A), None, None) == awq.ERR_SHAPE    # exactness limit

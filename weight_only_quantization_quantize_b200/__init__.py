@@ -10,7 +10,8 @@ Functions (names follow the C ABI):
   act_stats(xcal)                  -> m float32 [K]
   compute_scales(m)                -> s float16 [K]
   quantize_pack(W, s)              -> (Q int32 [K/8,N], scales float16 [K/128,N], zeros int32 [K/128,N/8])
-  w4a16_gemv(X, s, Q, scales, zeros)   X [1,K] -> Y [1,N]
+  quantize_pack(W, s, zero_point=False) -> (Q, scales, None)   symmetric grid, zero point 8
+  w4a16_gemv(X, s, Q, scales, zeros)   X [1,K] -> Y [1,N]   (zeros None: symmetric weights)
   w4a16_gemm(X, s, Q, scales, zeros)   X [M,K] -> Y [M,N]
 """
 from __future__ import annotations
@@ -38,7 +39,8 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_ARCH, ERR_CUDA, ERR_TIMEO
 # exported symbols, in declaration order of include/awq_b200.h
 SYMBOLS = (
     "awq_status_string", "awq_abi_version", "awq_act_stats", "awq_compute_scales",
-    "awq_quantize_pack", "awq_w4a16_gemv_workspace_size", "awq_w4a16_gemv",
+    "awq_quantize_pack", "awq_quantize_pack_symmetric", "awq_w4a16_gemv_workspace_size",
+    "awq_w4a16_gemv",
     "awq_w4a16_gemm_workspace_size", "awq_w4a16_gemm", "awq_w4a16_gemm_noalloc",
 )
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -70,6 +72,7 @@ def lib() -> ctypes.CDLL:
         L.awq_act_stats.argtypes = [P, I64, I64, P, P, P]
         L.awq_compute_scales.argtypes = [P, I64, P, P, P]
         L.awq_quantize_pack.argtypes = [P, P, I64, I64, P, P, P, P, P]
+        L.awq_quantize_pack_symmetric.argtypes = [P, P, I64, I64, P, P, P, P]
         L.awq_w4a16_gemv_workspace_size.argtypes = [I64, I64]
         L.awq_w4a16_gemv_workspace_size.restype = SZ
         L.awq_w4a16_gemv.argtypes = [P, P, P, P, P, I64, I64, P, P, SZ, P, P]
@@ -78,7 +81,8 @@ def lib() -> ctypes.CDLL:
         L.awq_w4a16_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, SZ, P, P]
         L.awq_w4a16_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P]
         for name in ("awq_act_stats", "awq_compute_scales", "awq_quantize_pack",
-                     "awq_w4a16_gemv", "awq_w4a16_gemm", "awq_w4a16_gemm_noalloc"):
+                     "awq_quantize_pack_symmetric", "awq_w4a16_gemv", "awq_w4a16_gemm",
+                     "awq_w4a16_gemm_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -152,8 +156,13 @@ def compute_scales(m: torch.Tensor, status: torch.Tensor | None = None) -> torch
     return s
 
 
-def quantize_pack(W: torch.Tensor, s: torch.Tensor, status: torch.Tensor | None = None, out=None):
-    """Fold s into W, 4-bit asymmetric group-128 quantization, packed int32."""
+def quantize_pack(W: torch.Tensor, s: torch.Tensor, status: torch.Tensor | None = None, out=None,
+                  zero_point: bool = True):
+    """Fold s into W, 4-bit group-128 quantization, packed int32.
+
+    zero_point=True: asymmetric grid with a per-group zero point (Q, scales, zeros).
+    zero_point=False: symmetric grid, zero point 8, no zeros tensor (Q, scales, None).
+    """
     _need(W, torch.float16, 2, "W")
     _need(s, torch.float16, 1, "s")
     K, N = W.shape
@@ -161,12 +170,18 @@ def quantize_pack(W: torch.Tensor, s: torch.Tensor, status: torch.Tensor | None 
     if out is None:
         Q = torch.empty(K // 8, N, dtype=torch.int32, device=dev)
         sc = torch.empty(max(K // GROUP_SIZE, 1), N, dtype=torch.float16, device=dev)
-        z = torch.empty(max(K // GROUP_SIZE, 1), max(N // 8, 1), dtype=torch.int32, device=dev)
+        z = (torch.empty(max(K // GROUP_SIZE, 1), max(N // 8, 1), dtype=torch.int32, device=dev)
+             if zero_point else None)
     else:
         Q, sc, z = out
     with torch.cuda.device(dev):
-        _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), K, N, _ptr(Q), _ptr(sc), _ptr(z),
-                                       _ptr(status), _stream(W)), "awq_quantize_pack")
+        if zero_point:
+            _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), K, N, _ptr(Q), _ptr(sc), _ptr(z),
+                                           _ptr(status), _stream(W)), "awq_quantize_pack")
+        else:
+            _check(lib().awq_quantize_pack_symmetric(_ptr(W), _ptr(s), K, N, _ptr(Q), _ptr(sc),
+                                                     _ptr(status), _stream(W)),
+                   "awq_quantize_pack_symmetric")
     return Q, sc, z
 
 

@@ -114,10 +114,12 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                         int64_t N, uint16_t *Y, void *ws, size_t ws_bytes, int32_t *dev_status,
                         awq_stream_t stream)
 {
-    if (!X || !s || !Q || !scales || !zeros || !Y) return AWQ_ERR_NULL;
+    // zeros == NULL: symmetric weights (zero point 8)
+    if (!X || !s || !Q || !scales || !Y) return AWQ_ERR_NULL;
     if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
-        !aligned16(Y) || (ws && !aligned16(ws)) || (dev_status && !aligned4(dev_status)))
+    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) ||
+        (zeros && !aligned16(zeros)) || !aligned16(Y) || (ws && !aligned16(ws)) ||
+        (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
     const size_t need = workspace_bytes(M, K);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return AWQ_ERR_WORKSPACE;
@@ -200,10 +202,10 @@ awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int3
                                 const uint16_t *scales, const int32_t *zeros, int64_t M,
                                 int64_t K, int64_t N, const uint16_t *Y, const int32_t *dev_status)
 {
-    if (!X || !s || !Q || !scales || !zeros || !Y) return AWQ_ERR_NULL;
+    if (!X || !s || !Q || !scales || !Y) return AWQ_ERR_NULL;
     if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
-        !aligned16(Y) || (dev_status && !aligned4(dev_status)))
+    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) ||
+        (zeros && !aligned16(zeros)) || !aligned16(Y) || (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
     return AWQ_OK;
 }
@@ -265,15 +267,19 @@ awq_status_t awq_compute_scales(const float *m, int64_t K, uint16_t *s, int32_t 
                                                 static_cast<cudaStream_t>(stream)));
 }
 
-awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
-                               int32_t *Q, uint16_t *scales, int32_t *zeros, int32_t *dev_status,
-                               awq_stream_t stream)
+}  // extern "C"
+
+namespace {
+// Both quantizers: zeros == NULL selects the symmetric grid, for which the
+// kernel writes no zero points.
+awq_status_t quantize_pack_any(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N, int32_t *Q,
+                               uint16_t *scales, int32_t *zeros, int32_t *dev_status, awq_stream_t stream)
 {
-    if (!W || !s || !Q || !scales || !zeros) return AWQ_ERR_NULL;
+    if (!W || !s || !Q || !scales) return AWQ_ERR_NULL;
     if (K < kGroup || K % kGroup != 0 || K > AWQ_MAX_K || N < 8 || N % 8 != 0 || N > AWQ_MAX_N)
         return AWQ_ERR_SHAPE;
-    if (!aligned16(W) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) || !aligned16(zeros) ||
-        (dev_status && !aligned4(dev_status)))
+    if (!aligned16(W) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) ||
+        (zeros && !aligned16(zeros)) || (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
     int sms = 0;
     awq_status_t e = device_ready(&sms);
@@ -285,6 +291,24 @@ awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, 
     return from_cuda(awq::launch_quantize_pack(tmW, reinterpret_cast<const __half *>(s), static_cast<int>(K),
                                                static_cast<int>(N), Q, reinterpret_cast<__half *>(scales),
                                                zeros, dev_status, sms, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+awq_status_t awq_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                               int32_t *Q, uint16_t *scales, int32_t *zeros, int32_t *dev_status,
+                               awq_stream_t stream)
+{
+    if (!zeros) return AWQ_ERR_NULL;
+    return quantize_pack_any(W, s, K, N, Q, scales, zeros, dev_status, stream);
+}
+
+awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                                         int32_t *Q, uint16_t *scales, int32_t *dev_status,
+                                         awq_stream_t stream)
+{
+    return quantize_pack_any(W, s, K, N, Q, scales, nullptr, dev_status, stream);
 }
 
 size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N)

@@ -151,6 +151,27 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- zero points
+// Symmetric weights ("Zero-Point Quantization" with zero_point False) come
+// without a zeros tensor: their zero point is 8 in every nibble.  Producers
+// copy these constant words in its place, so the consumers are the same for
+// both kinds of weights.
+__device__ __align__(16) const uint32_t kSymmetricZeroWords[32] = {
+    0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u,
+    0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u,
+    0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u,
+    0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u,
+    0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u};
+
+// Address of zero-point word `wi` of group g (zeros is [G, N/8]), or of a
+// constant word of 8s when zeros is NULL (`slot` < 32 picks one of them).
+__device__ __forceinline__ const int32_t *zero_word_src(const int32_t *zeros, int g, int words_per_row,
+                                                        int wi, int slot)
+{
+    return zeros ? zeros + static_cast<size_t>(g) * words_per_row + wi
+                 : reinterpret_cast<const int32_t *>(kSymmetricZeroWords) + (slot & 31);
+}
+
 // ---------------------------------------------------------------- cluster / DSMEM
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {

@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wi = n0 / 8 + lane;
             const bool in_z = wi < p.N / 8;
             cp_async_4(meta + 512 + 4 * lane,
-                       p.zeros + static_cast<size_t>(g) * (p.N / 8) + (in_z ? wi : 0), in_z ? 4u : 0u);
+                       zero_word_src(p.zeros, g, p.N / 8, in_z ? wi : 0, lane), in_z ? 4u : 0u);
             cp_async_arrive_noinc(&full_load[st]);
         }
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);

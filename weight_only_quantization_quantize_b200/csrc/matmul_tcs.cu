@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int wi = n0 / 8 + (lane - 16);
                 const bool in = wi < p.N / 8;
                 cp_async_4(meta + 256 + 4 * (lane - 16),
-                           p.zeros + static_cast<size_t>(g) * (p.N / 8) + (in ? wi : 0), in ? 4u : 0u);
+                           zero_word_src(p.zeros, g, p.N / 8, in ? wi : 0, lane), in ? 4u : 0u);
             }
             cp_async_arrive_noinc(&full_load[st]);
         }

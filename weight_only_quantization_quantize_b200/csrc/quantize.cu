@@ -1,5 +1,8 @@
 // quantize.cu -- activation statistics, per-channel scales, and the fused
-// fold + asymmetric 4-bit group quantization + packing (sm_100a).
+// fold + 4-bit group quantization + packing (sm_100a): asymmetric with a
+// per-group zero point, or symmetric ("Zero-Point Quantization" with
+// zero_point False: step = fp16(max(max|w'|, 1e-5) / 7), zero point 8, no
+// zeros tensor written).
 //
 // Sources: lansai AWQ explainer (ai.lansai.wang/107648), "AWQ 的四步链路"
 // (collect input magnitudes, Y = (X/s)(sW), quantize and pack by bits/group/
@@ -386,13 +389,17 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
                 a = 0.0f;
                 b = 0.0f;
             }
-            float r = __fsub_rn(a, b);
+            // asymmetric: step from the range, zero point from the minimum;
+            // symmetric (no zeros tensor): step from the largest magnitude over
+            // 7 levels, zero point 8, i.e. codes clamp(rint(w'/step), -8, 7) + 8
+            const bool symmetric = p.zeros == nullptr;
+            float r = symmetric ? fmaxf(fabsf(a), fabsf(b)) : __fsub_rn(a, b);
             if (r < 1e-5f) r = 1e-5f;
-            uint16_t bits = __half_as_ushort(__float2half_rn(__fdiv_rn(r, 15.0f)));
+            uint16_t bits = __half_as_ushort(__float2half_rn(__fdiv_rn(r, symmetric ? 7.0f : 15.0f)));
             if ((bits & 0x7FFF) == 0) bits = 1;  // never a zero step
             const float sf = __half2float(__ushort_as_half(bits));
             const float rsf = __frcp_rn(sf);
-            float zf = rint_quotient(-b, sf, rsf);
+            float zf = symmetric ? 8.0f : rint_quotient(-b, sf, rsf);
             zf = fminf(fmaxf(zf, 0.0f), 15.0f);
             const int z = static_cast<int>(zf);
             // codes are monotone in w', so the extremes decide whether any clamps
@@ -406,7 +413,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_pack_kernel(const __gri
         }
         named_bar_sync(bar_id, 256);  // column parameters ready
 
-        if (tid < kQTileN / 8 && n0 + 8 * tid < p.N) {
+        if (p.zeros != nullptr && tid < kQTileN / 8 && n0 + 8 * tid < p.N) {
             uint32_t zw = 0;
 #pragma unroll
             for (int c = 0; c < 8; ++c) zw |= static_cast<uint32_t>(sm.zc[8 * tid + c] & 15) << (4 * c);
