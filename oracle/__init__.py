@@ -60,10 +60,11 @@ def configure(lib):
     lib.awq_oracle_quantize_pack.argtypes = [P, P, I64, I64, P, P, P]
     lib.awq_oracle_quantize_pack_symmetric.argtypes = [P, P, I64, I64, P, P]
     lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
+    lib.awq_oracle_fold_inverse_scale.argtypes = [P, I64, I64, P, P]
     lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
     for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
               lib.awq_oracle_quantize_pack, lib.awq_oracle_quantize_pack_symmetric,
-              lib.awq_oracle_dequant, lib.awq_oracle_matmul):
+              lib.awq_oracle_dequant, lib.awq_oracle_matmul, lib.awq_oracle_fold_inverse_scale):
         f.restype = ctypes.c_int
     return lib
 
@@ -163,6 +164,25 @@ def quantize_pack(W, s, zero_point: bool = True):
     return Q, sc.view(np.float16), z
 
 
+def fold_inverse_scale(a, s) -> np.ndarray:
+    """out = fp16(a / s) per input channel (1/s folded into the preceding operator).
+
+    Lansai explainer, four-step chain: (X/s)(sW); a is [K] (a normalisation
+    weight) or [rows, K] (activations).  Returns float16 of a's shape.
+    """
+    av = _h(a)
+    shape = av.shape
+    a2 = av.reshape(1, -1) if av.ndim == 1 else av
+    sv = _h(s)
+    rows, K = a2.shape
+    if sv.shape != (K,):
+        raise ValueError("s must have shape [K]")
+    out = np.empty((rows, K), dtype=np.uint16)
+    _check(_load().awq_oracle_fold_inverse_scale(_p(np.ascontiguousarray(a2)), rows, K, _p(sv), _p(out)),
+           "fold_inverse_scale")
+    return out.reshape(shape).view(np.float16)
+
+
 def _zeros_ptr(zeros):
     """(array, pointer) for a zeros tensor; None (symmetric weights) is NULL."""
     if zeros is None:
@@ -190,13 +210,13 @@ def matmul(X, s, Q, scales, zeros, cols=None, precision: int = 64, nthreads: int
     Lansai explainer, four-step chain: Y = (X/s)(sW).  precision=64 computes
     everything in double; precision=32 is the dequantise-then-float-matmul
     (IEEE float division for X/s, float accumulation, k ascending, no FMA).
-    zeros=None: symmetric weights (z = 8).
+    zeros=None: symmetric weights (z = 8).  s=None: X already holds X/s.
     X: binary16 [M, K].  Returns float64 [M, len(cols)].
     """
     x = _h(X)
     if x.ndim == 1:
         x = x.reshape(1, -1)
-    sv = _h(s)
+    sv = None if s is None else _h(s)
     Q = np.ascontiguousarray(Q, dtype=np.int32)
     sc = _h(scales)
     z, zp = _zeros_ptr(zeros)
@@ -206,7 +226,7 @@ def matmul(X, s, Q, scales, zeros, cols=None, precision: int = 64, nthreads: int
         cols = np.arange(N, dtype=np.int64)
     cols = np.ascontiguousarray(cols, dtype=np.int64)
     Y = np.empty((M, cols.shape[0]), dtype=np.float64)
-    _check(_load().awq_oracle_matmul(_p(x), _p(sv), _p(Q), _p(sc), zp, M, K, N, _p(cols),
+    _check(_load().awq_oracle_matmul(_p(x), None if sv is None else _p(sv), _p(Q), _p(sc), zp, M, K, N, _p(cols),
                                      cols.shape[0], _p(Y), int(precision), int(nthreads)),
            "matmul")
     return Y

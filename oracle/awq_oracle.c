@@ -282,6 +282,32 @@ int awq_oracle_quantize_pack_symmetric(const uint16_t *W, const uint16_t *s, int
 }
 
 /* ---------------------------------------------------------------------------
+ * Folding 1/s into the preceding operator -- [P2] four-step chain: Y = XW is
+ * rewritten as (X/s)(sW); the X/s side can be carried by the operator that
+ * produces X (a normalisation weight, or the activations themselves), so the
+ * matmul receives X' = X/s.
+ * READING: out[r, k] = binary16_RNE(float(a[r, k]) / float(s_k)) with one IEEE
+ * float division, for rows x K inputs a (a normalisation weight is rows = 1).
+ * ------------------------------------------------------------------------ */
+int awq_oracle_fold_inverse_scale(const uint16_t *a, int64_t rows, int64_t K, const uint16_t *s,
+                                  uint16_t *out)
+{
+    if (!a || !s || !out)
+        return OR_ERR_NULL;
+    if (rows < 1 || K < 1)
+        return OR_ERR_SHAPE;
+    for (int64_t k = 0; k < K; ++k) {
+        float sk = h2f(s[k]);
+        if (!isfinite(sk) || !(sk > 0.0f))
+            return OR_ERR_NONFINITE;
+    }
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = f2h(h2f(a[r * K + k]) / h2f(s[k]));
+    return OR_OK;
+}
+
+/* ---------------------------------------------------------------------------
  * Step 7 -- dequantization (the pages' "伪量化" fake quantization: simulate the
  * low-bit weights in floating point).  w_hat[k,n] = (q - z) * scale_h, which
  * is exact in double; zeros == NULL means the symmetric grid (z = 8).  Output
@@ -318,7 +344,7 @@ int awq_oracle_dequant(const int32_t *Q, const uint16_t *scales, const int32_t *
 /* ---------------------------------------------------------------------------
  * Step 8 -- Y = (X / s) . dequant(Q), the plain definition (no blocking, k
  * ascending), for a chosen list of output columns.  [P2] four-step chain:
- * Y = (X/s)(sW).
+ * Y = (X/s)(sW).  s == NULL: X already holds X/s (1/s folded upstream), x' = x.
  *   precision 64: x' = x / s, w_hat and the sum all in double.
  *   precision 32: x' = float(x) / float(s) (IEEE float division), w_hat =
  *                 float(q - z) * float(scale_h) (exact), float accumulation
@@ -348,8 +374,9 @@ static void *mm_worker(void *arg)
                 double acc = 0.0;
                 for (int64_t k = 0; k < jb->K; ++k) {
                     int64_t g = k / GROUP;
-                    double xp = awq_oracle_half_to_double(jb->X[mrow * jb->K + k]) /
-                                awq_oracle_half_to_double(jb->s[k]);
+                    double xp = awq_oracle_half_to_double(jb->X[mrow * jb->K + k]);
+                    if (jb->s)
+                        xp = xp / awq_oracle_half_to_double(jb->s[k]);
                     double wh = (double)(code_at(jb->Q, jb->N, k, n) -
                                          zero_at(jb->zeros, jb->N, g, n)) *
                                 awq_oracle_half_to_double(jb->scales[g * jb->N + n]);
@@ -360,7 +387,9 @@ static void *mm_worker(void *arg)
                 float acc = 0.0f;
                 for (int64_t k = 0; k < jb->K; ++k) {
                     int64_t g = k / GROUP;
-                    float xp = h2f(jb->X[mrow * jb->K + k]) / h2f(jb->s[k]);
+                    float xp = h2f(jb->X[mrow * jb->K + k]);
+                    if (jb->s)
+                        xp = xp / h2f(jb->s[k]);
                     float wh = (float)(code_at(jb->Q, jb->N, k, n) -
                                        zero_at(jb->zeros, jb->N, g, n)) *
                                h2f(jb->scales[g * jb->N + n]);
@@ -379,7 +408,8 @@ int awq_oracle_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                       int64_t N, const int64_t *cols, int64_t ncols, double *Y,
                       int precision, int nthreads)
 {
-    if (!X || !s || !Q || !scales || !cols || !Y)   /* zeros may be NULL (symmetric) */
+    /* zeros may be NULL (symmetric weights); s may be NULL (X already holds X/s) */
+    if (!X || !Q || !scales || !cols || !Y)
         return OR_ERR_NULL;
     if (M < 1 || K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0 || ncols < 1)
         return OR_ERR_SHAPE;

@@ -37,6 +37,7 @@ MUTANTS = {
     "symmetric levels round half away": ("float level = nearbyintf(w / sf);", "float level = roundf(w / sf);"),
     "symmetric codes offset by 7": ("int32_t q = (int32_t)level + 8;", "int32_t q = (int32_t)level + 7;"),
     "symmetric range without absolute value": ("if (fabsf(w) > amax) amax = fabsf(w);", "if (w > amax) amax = w;"),
+    "fold multiplies by s": ("f2h(h2f(a[r * K + k]) / h2f(s[k]))", "f2h(h2f(a[r * K + k]) * h2f(s[k]))"),
     "missing zeros read as zero": ("if (!zeros)\n        return 8;", "if (!zeros)\n        return 0;"),
 }
 

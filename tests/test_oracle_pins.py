@@ -511,3 +511,52 @@ def test_symmetric_matmul_lossless_grid_equals_plain_xw(M, K, N):
     Y = oracle.matmul(X, s.astype(np.float16), Q, sc, None, precision=64)
     ref = X.astype(np.float64) @ W
     assert np.max(np.abs(Y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+# --------------------------------------------------------------------------
+# 1/s folded into the preceding operator (lansai four-step chain: (X/s)(sW))
+# --------------------------------------------------------------------------
+def test_fold_inverse_scale_equals_numpy_float_division():
+    rng = np.random.default_rng(31)
+    K = 4096
+    a = (rng.standard_normal((3, K)) * rng.uniform(0.01, 30, K)).astype(np.float16)
+    s = rng.uniform(0.05, 20.0, K).astype(np.float16)
+    got = oracle.fold_inverse_scale(a, s)
+    ref = (a.astype(np.float32) / s.astype(np.float32)).astype(np.float16)   # IEEE float, one RNE
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+    g1 = oracle.fold_inverse_scale(a[0], s)                                # a norm weight [K]
+    assert g1.shape == (K,) and np.array_equal(g1.view(np.uint16), got[0].view(np.uint16))
+
+
+def test_fold_inverse_scale_closed_forms_and_errors():
+    rng = np.random.default_rng(32)
+    K = 256
+    a = rng.standard_normal((2, K)).astype(np.float16)
+    assert np.array_equal(oracle.fold_inverse_scale(a, np.ones(K, np.float16)).view(np.uint16),
+                          a.view(np.uint16))
+    p2 = 2.0 ** rng.integers(-3, 4, K)
+    out = oracle.fold_inverse_scale(a, p2.astype(np.float16)).astype(np.float64)
+    assert np.array_equal(out, a.astype(np.float64) / p2)                  # exact, no underflow here
+    bad = np.ones(K, np.float16)
+    bad[7] = 0
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.fold_inverse_scale(a, bad)
+    assert e.value.code == oracle.ERR_NONFINITE
+
+
+def test_matmul_without_s_reads_prescaled_activations():
+    L = synth.make_layer(1, 0, M=4, K=512, N=64, R=32)
+    s = oracle.compute_scales(oracle.act_stats(L.Xcal.numpy()))
+    Q, sc, z = oracle.quantize_pack(L.W.numpy(), s)
+    X = L.X.numpy()
+    # no s is the same as s = 1 (division by one is exact)
+    ones = np.ones(512, np.float16)
+    for prec in (64, 32):
+        assert np.array_equal(oracle.matmul(X, None, Q, sc, z, precision=prec),
+                              oracle.matmul(X, ones, Q, sc, z, precision=prec))
+    # power-of-two s: X/s is exact in binary16, so folding it upstream changes nothing
+    rng = np.random.default_rng(33)
+    p2 = (2.0 ** rng.integers(-2, 3, 512)).astype(np.float16)
+    Xp = oracle.fold_inverse_scale(X, p2)
+    assert np.array_equal(oracle.matmul(Xp, None, Q, sc, z, precision=64),
+                          oracle.matmul(X, p2, Q, sc, z, precision=64))
