@@ -247,6 +247,7 @@ def run_ours(args, rank, world, device):
         extra["small_batch_13b_m48"] = run_small_batch(awq, device, peaks)
         extra["quantize_7b_layer_symmetric"] = run_quantize(awq, device, layers, peaks, zero_point=False)
         extra["decode_7b_symmetric"] = run_decode_symmetric(awq, device, peaks, nlayers)
+        extra["decode_7b_prescaled"] = run_decode_symmetric(awq, device, peaks, nlayers, prescaled=True)
 
     cpu = run_cpu_baseline(rank, world) if rank == 0 else None
     return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, launches=launches,
@@ -379,16 +380,27 @@ def run_small_batch(awq, device, peaks, M=48, reps=10):
             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "includes": "X/s pre-pass + 4 GEMMs"}
 
 
-def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5):
-    """The decode step on symmetric weights (zeros = NULL), timed like the headline.
+def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5, prescaled=False):
+    """A decode-step variant, timed like the headline.
 
-    Algorithmic bytes: 0.5 B per weight + 2 B per 128 weights (no zero points)."""
+    prescaled=False: symmetric weights (zeros = NULL); algorithmic bytes 0.5 B
+    per weight + 2 B per 128 weights (no zero points).
+    prescaled=True: the headline's asymmetric weights with 1/s folded upstream
+    (X already holds X/s, s = NULL); 0.5195 B per weight."""
     wl = synth.WORKLOADS[WORKLOAD_ID]
-    layers = build_layers(awq, nlayers, device, zero_point=False)
+    layers = build_layers(awq, nlayers, device, zero_point=prescaled)
+    if prescaled:
+        for lp in layers:
+            for p in lp:
+                p["X"] = awq.fold_inverse_scale(p["X"], p["s"])
+        torch.cuda.synchronize()
 
     def step(i):
         for p in layers[i % nlayers]:
-            awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], None, out=p["Y"])
+            if prescaled:
+                awq.w4a16_gemv(p["X"], None, p["Q"], p["sc"], p["z"], out=p["Y"])
+            else:
+                awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], None, out=p["Y"])
 
     for i in range(warmup):
         step(i)
@@ -406,11 +418,13 @@ def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     del g, layers
-    wbytes = sum(K * N * (0.5 + 2 / 128) for K, N, _ in wl.shapes)
+    per_weight = BYTES_PER_WEIGHT if prescaled else 0.5 + 2 / 128
+    wbytes = sum(K * N * per_weight for K, N, _ in wl.shapes)
     gbs = wbytes * steps / (ms * 1e-3) / 1e9
     return {"ms_per_step": round(ms / steps, 5), "weight_gbs": round(gbs, 1),
             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-            "bytes": "0.5 B/weight codes + fp16 step per 128 weights; no zero points",
+            "bytes": ("0.5195 B/weight (codes, steps, zeros); X already divided by s" if prescaled
+                      else "0.5 B/weight codes + fp16 step per 128 weights; no zero points"),
             "l2": f"{nlayers} distinct layers rotated", "timing": "CUDA graph, CUDA events"}
 
 

@@ -64,7 +64,7 @@ extern "C" {
 #define AWQ_MAX_K 262144
 #define AWQ_MAX_N 1048576
 #define AWQ_MAX_M 1048576
-#define AWQ_ABI_VERSION 2  /* 2: symmetric weights (quantize + NULL zeros) */
+#define AWQ_ABI_VERSION 3  /* 2: symmetric weights; 3: 1/s folded upstream */
 
 typedef enum {
     AWQ_OK = 0,
@@ -168,6 +168,10 @@ AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16
  * internally (register-fed tensor cores for M < 64, tcgen05/TMEM for M >= 64).
  *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack;
  *   zeros = NULL for weights from awq_quantize_pack_symmetric (zero point 8).
+ *   s = NULL when X already holds X/s (1/s folded into the operator that
+ *   produced X, e.g. by awq_fold_inverse_scale): X is then used as it is, and
+ *   with X = awq_fold_inverse_scale(X, s) the result equals, bit for bit,
+ *   the call with the original X and s.
  * Workspace: caller-owned device memory of at least *_workspace_size() bytes
  * (may be NULL when that size is 0); it holds X / s and is overwritten.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
@@ -180,6 +184,21 @@ AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16
  * Ordinary kernels, copies and awq_quantize_pack complete before any
  * dependent starts, so writing the weights with them is safe.
  */
+/*
+ * Fold 1/s upstream -- lansai explainer, "AWQ 的四步链路": Y = XW = (X/s)(sW),
+ * with the X/s side carried by the operator that produces X (a normalisation
+ * weight: rows = 1; or activations divided once for several projections).
+ *   out[r, k] = binary16_RNE(float(a[r, k]) / float(s_k))   (IEEE division)
+ * the same operations the matmul applies to X when it is given s.
+ *   a    binary16 [rows, K], 1 <= rows <= AWQ_MAX_M, K % 8 == 0
+ *   s    binary16 [K] (> 0);  out binary16 [rows, K] (output, not aliasing a)
+ * Device errors: AWQ_ERR_NONFINITE if some s_k is NaN/Inf or <= 0 (out is
+ * still written).
+ */
+AWQ_API awq_status_t awq_fold_inverse_scale(const uint16_t *a, int64_t rows, int64_t K,
+                                    const uint16_t *s, uint16_t *out, int32_t *dev_status,
+                                    awq_stream_t stream);
+
 AWQ_API size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N);
 AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                             const uint16_t *scales, const int32_t *zeros, int64_t K, int64_t N,

@@ -52,7 +52,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.awq_abi_version() == 2
+    assert L.awq_abi_version() == 3
     for code, name in awq.STATUS.items():
         assert awq.status_string(code).startswith(name)
     assert awq.status_string(99) == "AWQ_ERR_UNKNOWN"
@@ -76,6 +76,9 @@ def test_matmul_validation(L):
     assert gemm(L, z=0, K=100) == awq.ERR_SHAPE
     assert gemm(L, z=0, Y=0) == awq.ERR_NULL
     assert gemm(L, z=MIS) == awq.ERR_ALIGN
+    # s = NULL is legal too (X already holds X/s)
+    assert gemm(L, s=0, N=12) == awq.ERR_SHAPE
+    assert gemm(L, s=MIS) == awq.ERR_ALIGN
     assert gemm(L, Y=0) == awq.ERR_NULL
     assert gemm(L, K=100) == awq.ERR_SHAPE            # K % 128
     assert gemm(L, K=0) == awq.ERR_SHAPE
@@ -90,7 +93,7 @@ def test_matmul_validation(L):
     assert gemm(L, wsb=100) == awq.ERR_WORKSPACE
     r = L.awq_w4a16_gemv(P(A), P(A), P(A), P(A), P(A), 4096, 4097, P(A), None, 0, None, None)
     assert r == awq.ERR_SHAPE
-    r = L.awq_w4a16_gemv(P(A), P(0), P(A), P(A), P(A), 4096, 4096, P(A), None, 0, None, None)
+    r = L.awq_w4a16_gemv(P(0), P(A), P(A), P(A), P(A), 4096, 4096, P(A), None, 0, None, None)
     assert r == awq.ERR_NULL
 
 
@@ -114,6 +117,13 @@ def test_quantize_and_stats_validation(L):
     assert st(P(A), 16, 1020, P(A), None, None) == awq.ERR_SHAPE
     assert st(P(0), 16, 1024, P(A), None, None) == awq.ERR_NULL
     assert st(P(A), 16, 1024, P(MIS), None, None) == awq.ERR_ALIGN
+    fo = L.awq_fold_inverse_scale
+    assert fo(P(0), 1, 4096, P(A), P(A), None, None) == awq.ERR_NULL
+    assert fo(P(A), 1, 4096, P(0), P(A), None, None) == awq.ERR_NULL
+    assert fo(P(A), 1, 4096, P(A), P(0), None, None) == awq.ERR_NULL
+    assert fo(P(A), 0, 4096, P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert fo(P(A), 1, 4100, P(A), P(A), None, None) == awq.ERR_SHAPE
+    assert fo(P(A), 1, 4096, P(A), P(MIS), None, None) == awq.ERR_ALIGN
     cs = L.awq_compute_scales
     assert cs(P(A), 0, P(A), None, None) == awq.ERR_SHAPE
     assert cs(P(A), 16, P(0), None, None) == awq.ERR_NULL

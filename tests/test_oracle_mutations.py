@@ -32,7 +32,7 @@ MUTANTS = {
                                         "((uint32_t)Q[(k % 8) * N + n] >> (4 * ((k / 8) % 8)))"),
     "subnormal exponent off by one": ("v = ldexp((double)f, -24);", "v = ldexp((double)f, -25);"),
     "binary16 ties rounded away": ("double n = nearbyint(ldexp(a, -q));", "double n = round(ldexp(a, -q));"),
-    "activation multiplied by s": ("jb->X[mrow * jb->K + k]) /", "jb->X[mrow * jb->K + k]) *"),
+    "activation multiplied by s": ("xp = xp / ", "xp = xp * "),
     "symmetric step from max/8": ("f2h(amax / 7.0f)", "f2h(amax / 8.0f)"),
     "symmetric levels round half away": ("float level = nearbyintf(w / sf);", "float level = roundf(w / sf);"),
     "symmetric codes offset by 7": ("int32_t q = (int32_t)level + 8;", "int32_t q = (int32_t)level + 7;"),

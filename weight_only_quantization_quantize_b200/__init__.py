@@ -11,7 +11,9 @@ Functions (names follow the C ABI):
   compute_scales(m)                -> s float16 [K]
   quantize_pack(W, s)              -> (Q int32 [K/8,N], scales float16 [K/128,N], zeros int32 [K/128,N/8])
   quantize_pack(W, s, zero_point=False) -> (Q, scales, None)   symmetric grid, zero point 8
-  w4a16_gemv(X, s, Q, scales, zeros)   X [1,K] -> Y [1,N]   (zeros None: symmetric weights)
+  fold_inverse_scale(a, s)         -> fp16(a / s), a [K] or [rows,K] (1/s folded upstream)
+  w4a16_gemv(X, s, Q, scales, zeros)   X [1,K] -> Y [1,N]   (zeros None: symmetric weights;
+                                                             s None: X already holds X/s)
   w4a16_gemm(X, s, Q, scales, zeros)   X [M,K] -> Y [M,N]
 """
 from __future__ import annotations
@@ -39,7 +41,8 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_ARCH, ERR_CUDA, ERR_TIMEO
 # exported symbols, in declaration order of include/awq_b200.h
 SYMBOLS = (
     "awq_status_string", "awq_abi_version", "awq_act_stats", "awq_compute_scales",
-    "awq_quantize_pack", "awq_quantize_pack_symmetric", "awq_w4a16_gemv_workspace_size",
+    "awq_quantize_pack", "awq_quantize_pack_symmetric", "awq_fold_inverse_scale",
+    "awq_w4a16_gemv_workspace_size",
     "awq_w4a16_gemv",
     "awq_w4a16_gemm_workspace_size", "awq_w4a16_gemm", "awq_w4a16_gemm_noalloc",
 )
@@ -73,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.awq_compute_scales.argtypes = [P, I64, P, P, P]
         L.awq_quantize_pack.argtypes = [P, P, I64, I64, P, P, P, P, P]
         L.awq_quantize_pack_symmetric.argtypes = [P, P, I64, I64, P, P, P, P]
+        L.awq_fold_inverse_scale.argtypes = [P, I64, I64, P, P, P, P]
         L.awq_w4a16_gemv_workspace_size.argtypes = [I64, I64]
         L.awq_w4a16_gemv_workspace_size.restype = SZ
         L.awq_w4a16_gemv.argtypes = [P, P, P, P, P, I64, I64, P, P, SZ, P, P]
@@ -81,7 +85,8 @@ def lib() -> ctypes.CDLL:
         L.awq_w4a16_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, SZ, P, P]
         L.awq_w4a16_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, P]
         for name in ("awq_act_stats", "awq_compute_scales", "awq_quantize_pack",
-                     "awq_quantize_pack_symmetric", "awq_w4a16_gemv", "awq_w4a16_gemm",
+                     "awq_quantize_pack_symmetric", "awq_fold_inverse_scale", "awq_w4a16_gemv",
+                     "awq_w4a16_gemm",
                      "awq_w4a16_gemm_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -183,6 +188,22 @@ def quantize_pack(W: torch.Tensor, s: torch.Tensor, status: torch.Tensor | None 
                                                      _ptr(status), _stream(W)),
                    "awq_quantize_pack_symmetric")
     return Q, sc, z
+
+
+def fold_inverse_scale(a: torch.Tensor, s: torch.Tensor, status: torch.Tensor | None = None,
+                       out=None) -> torch.Tensor:
+    """out = fp16(a / s) per input channel; a is [K] (a norm weight) or [rows, K]."""
+    if a.dim() not in (1, 2):
+        raise ValueError("a must be [K] or [rows, K]")
+    a2 = a.view(1, -1) if a.dim() == 1 else a
+    _need(a2, torch.float16, 2, "a")
+    _need(s, torch.float16, 1, "s")
+    rows, K = a2.shape
+    o = torch.empty_like(a) if out is None else out
+    with torch.cuda.device(a.device):
+        _check(lib().awq_fold_inverse_scale(_ptr(a2), rows, K, _ptr(s), _ptr(o), _ptr(status),
+                                            _stream(a)), "awq_fold_inverse_scale")
+    return o
 
 
 def gemm_workspace_size(M: int, K: int, N: int) -> int:

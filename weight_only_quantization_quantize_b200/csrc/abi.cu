@@ -3,7 +3,8 @@
 // Host-side work only: argument validation (returned before any launch), a
 // one-time per-device architecture check, TMA descriptor encoding, workspace
 // accounting and the choice of tile path.  Every step of the computation runs
-// in the kernels of quantize.cu, matmul_small.cu and matmul_tc.cu.
+// in the kernels of quantize.cu, fold.cu, gemv.cu, matmul_small.cu,
+// matmul_tcs.cu and matmul_tc.cu.
 #include <cstdlib>
 #include <mutex>
 
@@ -114,10 +115,10 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                         int64_t N, uint16_t *Y, void *ws, size_t ws_bytes, int32_t *dev_status,
                         awq_stream_t stream)
 {
-    // zeros == NULL: symmetric weights (zero point 8)
-    if (!X || !s || !Q || !scales || !Y) return AWQ_ERR_NULL;
+    // zeros == NULL: symmetric weights (zero point 8); s == NULL: X holds X/s
+    if (!X || !Q || !scales || !Y) return AWQ_ERR_NULL;
     if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) ||
+    if (!aligned16(X) || (s && !aligned16(s)) || !aligned16(Q) || !aligned16(scales) ||
         (zeros && !aligned16(zeros)) || !aligned16(Y) || (ws && !aligned16(ws)) ||
         (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
@@ -202,9 +203,9 @@ awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int3
                                 const uint16_t *scales, const int32_t *zeros, int64_t M,
                                 int64_t K, int64_t N, const uint16_t *Y, const int32_t *dev_status)
 {
-    if (!X || !s || !Q || !scales || !Y) return AWQ_ERR_NULL;
+    if (!X || !Q || !scales || !Y) return AWQ_ERR_NULL;
     if (!matmul_shape_ok(M, K, N)) return AWQ_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(s) || !aligned16(Q) || !aligned16(scales) ||
+    if (!aligned16(X) || (s && !aligned16(s)) || !aligned16(Q) || !aligned16(scales) ||
         (zeros && !aligned16(zeros)) || !aligned16(Y) || (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
     return AWQ_OK;
@@ -309,6 +310,22 @@ awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16_t *s, i
                                          awq_stream_t stream)
 {
     return quantize_pack_any(W, s, K, N, Q, scales, nullptr, dev_status, stream);
+}
+
+awq_status_t awq_fold_inverse_scale(const uint16_t *a, int64_t rows, int64_t K, const uint16_t *s,
+                                    uint16_t *out, int32_t *dev_status, awq_stream_t stream)
+{
+    if (!a || !s || !out) return AWQ_ERR_NULL;
+    if (rows < 1 || rows > AWQ_MAX_M || K < 8 || K % 8 != 0 || K > AWQ_MAX_K) return AWQ_ERR_SHAPE;
+    if (!aligned16(a) || !aligned16(s) || !aligned16(out) || (dev_status && !aligned4(dev_status)))
+        return AWQ_ERR_ALIGN;
+    int sms = 0;
+    awq_status_t e = device_ready(&sms);
+    if (e != AWQ_OK) return e;
+    return from_cuda(awq::launch_fold_inverse_scale(reinterpret_cast<const __half *>(a), rows,
+                                                    static_cast<int>(K), reinterpret_cast<const __half *>(s),
+                                                    reinterpret_cast<__half *>(out), dev_status, sms,
+                                                    static_cast<cudaStream_t>(stream)));
 }
 
 size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N)

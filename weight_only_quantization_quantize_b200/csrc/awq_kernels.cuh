@@ -15,6 +15,10 @@ cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K,
                                  __half *scales, int32_t *zeros, int32_t *status, int num_sms,
                                  cudaStream_t st);
 
+// fold.cu -- out = fp16(a / s) per channel (1/s folded upstream)
+cudaError_t launch_fold_inverse_scale(const __half *a, int64_t rows, int K, const __half *s,
+                                      __half *out, int32_t *status, int num_sms, cudaStream_t st);
+
 // gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group
 struct GemvPlan {
     int splits;       // CTAs per cluster along K

@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                     if (valid[b]) {
                         const int k = (g_begin + gl[b]) * kGroup + c16 * 8;
                         xv[b] = __ldg(reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(tok[b]) * p.K + k));
-                        sv[b] = __ldg(reinterpret_cast<const uint4 *>(p.s + k));
+                        // s == NULL: X already holds X/s (division by 1 is exact)
+                        sv[b] = p.s ? __ldg(reinterpret_cast<const uint4 *>(p.s + k))
+                                    : make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
                     }
                 }
 #pragma unroll

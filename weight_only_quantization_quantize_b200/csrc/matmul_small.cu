@@ -80,7 +80,9 @@ __global__ void __launch_bounds__(256) prescale_kernel(const __half *__restrict_
     if (i >= chunks) return;
     const int kc = static_cast<int>(i % kchunks);
     const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(X) + i);
-    const uint4 sv = __ldg(reinterpret_cast<const uint4 *>(s) + kc);
+    // s == NULL: X already holds X/s; dividing by 1 leaves it bit for bit
+    const uint4 sv = s ? __ldg(reinterpret_cast<const uint4 *>(s) + kc)
+                       : make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
     reinterpret_cast<uint4 *>(Xp)[i] = prescale8(xv, sv);
 }
 
