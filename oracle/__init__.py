@@ -61,10 +61,13 @@ def configure(lib):
     lib.awq_oracle_quantize_pack_symmetric.argtypes = [P, P, I64, I64, P, P]
     lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
     lib.awq_oracle_fold_inverse_scale.argtypes = [P, I64, I64, P, P]
+    lib.awq_oracle_scales_alpha.argtypes = [P, I64, I, P]
+    lib.awq_oracle_scale_search.argtypes = [P, I64, I64, P, I64, P, P, P, I]
     lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
     for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
               lib.awq_oracle_quantize_pack, lib.awq_oracle_quantize_pack_symmetric,
-              lib.awq_oracle_dequant, lib.awq_oracle_matmul, lib.awq_oracle_fold_inverse_scale):
+              lib.awq_oracle_dequant, lib.awq_oracle_matmul, lib.awq_oracle_fold_inverse_scale,
+              lib.awq_oracle_scales_alpha, lib.awq_oracle_scale_search):
         f.restype = ctypes.c_int
     return lib
 
@@ -162,6 +165,37 @@ def quantize_pack(W, s, zero_point: bool = True):
     _check(_load().awq_oracle_quantize_pack(_p(w), _p(sv), K, N, _p(Q), _p(sc), _p(z)),
            "quantize_pack")
     return Q, sc.view(np.float16), z
+
+
+def scales_alpha(m, j: int) -> np.ndarray:
+    """s = normalised m^(j/8), j = 0..8, by the fixed sqrt/product chain (float16 [K]).
+
+    "Awq Quantization", "How AWQ Works" (the search over s); j = 4 is compute_scales.
+    """
+    m = np.ascontiguousarray(m, dtype=np.float32)
+    s = np.empty(m.shape[0], dtype=np.uint16)
+    _check(_load().awq_oracle_scales_alpha(_p(m), m.shape[0], int(j), _p(s)), "scales_alpha")
+    return s.view(np.float16)
+
+
+def scale_search(xcal, W, nthreads: int = 1):
+    """Grid search of alpha = j/8 minimising L(s) = ||Q(W s)(X/s) - X W||^2 on the calibration rows.
+
+    "Awq Quantization", "How AWQ Works"; lansai four-step chain, row "搜索缩放".
+    Returns (j_best, s_best float16 [K], losses float64 [9]).
+    """
+    x = _h(xcal)
+    w = _h(W)
+    R, K = x.shape
+    if w.shape[0] != K:
+        raise ValueError("W must be [K, N]")
+    N = w.shape[1]
+    losses = np.empty(9, dtype=np.float64)
+    s = np.empty(K, dtype=np.uint16)
+    jb = ctypes.c_int(-1)
+    _check(_load().awq_oracle_scale_search(_p(x), R, K, _p(w), N, _p(losses), _p(s),
+                                           ctypes.byref(jb), int(nthreads)), "scale_search")
+    return jb.value, s.view(np.float16), losses
 
 
 def fold_inverse_scale(a, s) -> np.ndarray:

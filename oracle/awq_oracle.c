@@ -150,6 +150,125 @@ int awq_oracle_compute_scales(const float *m, int64_t K, uint16_t *s)
 }
 
 /* ---------------------------------------------------------------------------
+ * Scale search (next row) -- [P3] "How AWQ Works": s is chosen to make
+ * L(s) = ||Q(W*s)(s^-1*X) - W*X|| small; [P2] four-step chain, row "搜索缩放"
+ * (evaluate the effect of different channel scalings on the reconstruction
+ * error).  The pages give neither the family nor the grid.
+ * READINGS:
+ *   family   s(alpha) = m^alpha normalised as in step 2 (alpha = 1/2 is step 2)
+ *   grid     alpha = j/8, j = 0..8, with m^alpha formed by one fixed chain of
+ *            IEEE double operations, so that every result is reproducible:
+ *              u = max(m, 1e-8), r1 = sqrt(u), r2 = sqrt(r1), r3 = sqrt(r2)
+ *              t = u                                   (j = 8)
+ *              t = 1 * [r1 if j&4] * [r2 if j&2] * [r3 if j&1]   (j < 8, in
+ *                  that order, left to right)
+ *            then c = sqrt(max t * min t) and s = binary16_RNE(t / c)
+ *   loss     L(j) = sum over calibration rows r and outputs n of
+ *            (Yq[r,n] - Y[r,n])^2 in double, Yq from the quantized layer
+ *            (steps 3-8 with s(j)) and Y = X W (both in double)
+ *   choice   the smallest j whose loss is the minimum
+ * ------------------------------------------------------------------------ */
+int awq_oracle_scales_alpha(const float *m, int64_t K, int j, uint16_t *s)
+{
+    if (!m || !s)
+        return OR_ERR_NULL;
+    if (K < 1 || j < 0 || j > 8)
+        return OR_ERR_SHAPE;
+    double *t = (double *)malloc(sizeof(double) * (size_t)K);
+    if (!t)
+        return OR_ERR_NULL;
+    double tmax = 0.0, tmin = INFINITY;
+    for (int64_t k = 0; k < K; ++k) {
+        if (!isfinite(m[k]) || m[k] < 0.0f) {
+            free(t);
+            return OR_ERR_NONFINITE;
+        }
+        double u = fmax((double)m[k], 1e-8);
+        double r1 = sqrt(u), r2 = sqrt(r1), r3 = sqrt(r2);
+        double v;
+        if (j == 8) {
+            v = u;
+        } else {
+            v = 1.0;
+            if (j & 4) v = v * r1;
+            if (j & 2) v = v * r2;
+            if (j & 1) v = v * r3;
+        }
+        t[k] = v;
+        if (v > tmax) tmax = v;
+        if (v < tmin) tmin = v;
+    }
+    double c = sqrt(tmax * tmin);
+    for (int64_t k = 0; k < K; ++k)
+        s[k] = awq_oracle_double_to_half(t[k] / c);
+    free(t);
+    return OR_OK;
+}
+
+int awq_oracle_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, int64_t N,
+                             int32_t *Q, uint16_t *scales, int32_t *zeros);
+int awq_oracle_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
+                      const uint16_t *scales, const int32_t *zeros, int64_t M, int64_t K,
+                      int64_t N, const int64_t *cols, int64_t ncols, double *Y,
+                      int precision, int nthreads);
+
+int awq_oracle_scale_search(const uint16_t *xcal, int64_t R, int64_t K, const uint16_t *W, int64_t N,
+                            double *losses, uint16_t *s_best, int *j_best, int nthreads)
+{
+    if (!xcal || !W || !losses || !s_best || !j_best)
+        return OR_ERR_NULL;
+    if (R < 1 || K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0)
+        return OR_ERR_SHAPE;
+    int rc = OR_ERR_NULL;
+    float *m = (float *)malloc(sizeof(float) * (size_t)K);
+    uint16_t *s = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)K);
+    int32_t *Q = (int32_t *)malloc(sizeof(int32_t) * (size_t)((K / 8) * N));
+    uint16_t *sc = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)((K / GROUP) * N));
+    int32_t *z = (int32_t *)malloc(sizeof(int32_t) * (size_t)((K / GROUP) * (N / 8)));
+    int64_t *cols = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    double *Yq = (double *)malloc(sizeof(double) * (size_t)(R * N));
+    double *Yr = (double *)malloc(sizeof(double) * (size_t)(R * N));
+    if (!m || !s || !Q || !sc || !z || !cols || !Yq || !Yr)
+        goto done;
+    rc = awq_oracle_act_stats(xcal, R, K, m);
+    if (rc != OR_OK)
+        goto done;
+    for (int64_t n = 0; n < N; ++n)
+        cols[n] = n;
+    /* Y = X W, the unquantized layer, in double (k ascending) */
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += awq_oracle_half_to_double(xcal[r * K + k]) * awq_oracle_half_to_double(W[k * N + n]);
+            Yr[r * N + n] = acc;
+        }
+    double best = INFINITY;
+    for (int j = 0; j <= 8; ++j) {
+        rc = awq_oracle_scales_alpha(m, K, j, s);
+        if (rc == OR_OK) rc = awq_oracle_quantize_pack(W, s, K, N, Q, sc, z);
+        if (rc == OR_OK) rc = awq_oracle_matmul(xcal, s, Q, sc, z, R, K, N, cols, N, Yq, 64, nthreads);
+        if (rc != OR_OK)
+            goto done;
+        double loss = 0.0;
+        for (int64_t i = 0; i < R * N; ++i) {
+            double d = Yq[i] - Yr[i];
+            loss += d * d;
+        }
+        losses[j] = loss;
+        if (loss < best) {
+            best = loss;
+            *j_best = j;
+            memcpy(s_best, s, sizeof(uint16_t) * (size_t)K);
+        }
+    }
+    rc = OR_OK;
+done:
+    free(m); free(s); free(Q); free(sc); free(z); free(cols); free(Yq); free(Yr);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
  * Steps 3-6 -- fold s into W, asymmetric 4-bit group quantization with a zero
  * point, and packing.
  *   [P2] four-step chain: enlarge the salient channels' weights (sW), then

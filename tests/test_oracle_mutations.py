@@ -38,6 +38,8 @@ MUTANTS = {
     "symmetric codes offset by 7": ("int32_t q = (int32_t)level + 8;", "int32_t q = (int32_t)level + 7;"),
     "symmetric range without absolute value": ("if (fabsf(w) > amax) amax = fabsf(w);", "if (w > amax) amax = w;"),
     "fold multiplies by s": ("f2h(h2f(a[r * K + k]) / h2f(s[k]))", "f2h(h2f(a[r * K + k]) * h2f(s[k]))"),
+    "alpha chain: 1/8 power from the square root": ("r3 = sqrt(r2);", "r3 = sqrt(r1);"),
+    "scale search keeps the largest loss": ("if (loss < best) {", "if (loss > best) {"),
     "missing zeros read as zero": ("if (!zeros)\n        return 8;", "if (!zeros)\n        return 0;"),
 }
 

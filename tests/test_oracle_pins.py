@@ -560,3 +560,64 @@ def test_matmul_without_s_reads_prescaled_activations():
     Xp = oracle.fold_inverse_scale(X, p2)
     assert np.array_equal(oracle.matmul(Xp, None, Q, sc, z, precision=64),
                           oracle.matmul(X, p2, Q, sc, z, precision=64))
+
+
+# --------------------------------------------------------------------------
+# scale search over alpha ("How AWQ Works": L(s); lansai chain row "搜索缩放")
+# --------------------------------------------------------------------------
+def test_alpha_scales_closed_forms():
+    rng = np.random.default_rng(41)
+    m = rng.uniform(0.01, 9.0, 512).astype(np.float32)
+    # j = 4 (alpha = 1/2) is the pinned single-point scale
+    assert np.array_equal(oracle.scales_alpha(m, 4).view(np.uint16), oracle.compute_scales(m).view(np.uint16))
+    # j = 0: every t is 1, so s is exactly 1
+    assert np.all(oracle.scales_alpha(m, 0) == 1.0)
+    # two levels 16 and 1: s = 16^(j/8) / 16^(j/16) = 2^(j/4) or its inverse;
+    # the double chain is within a few ulps of it, far from any binary16
+    # rounding boundary, so the stored value is 2^(+-j/4) rounded once
+    two = np.where(np.arange(64) % 2 == 0, 16.0, 1.0).astype(np.float32)
+    for j in range(9):
+        s = oracle.scales_alpha(two, j).astype(np.float64)
+        hi, lo = 2.0 ** (j / 4), 2.0 ** (-j / 4)
+        assert np.array_equal(s[0::2], np.full(32, float(np.float16(hi))))
+        assert np.array_equal(s[1::2], np.full(32, float(np.float16(lo))))
+    with pytest.raises(oracle.OracleError):
+        oracle.scales_alpha(m, 9)
+
+
+def _plain_rtn_loss(X16, W16):
+    """Output error of plain min-max RTN (s = 1), by the independent numpy quantizer."""
+    q, step, zero = _textbook_minmax_rtn(W16)
+    K, N = W16.shape
+    wh = (q - np.repeat(zero, 128, axis=0)) * np.repeat(step.astype(np.float64), 128, axis=0)
+    X = X16.astype(np.float64)
+    return float(np.sum((X @ wh - X @ W16.astype(np.float64)) ** 2))
+
+
+def test_scale_search_loss_grid_and_choice():
+    L = synth.make_layer(1, 0, M=1, K=256, N=64, R=32)
+    X, W = L.Xcal.numpy(), L.W.numpy()
+    j, s, losses = oracle.scale_search(X, W, nthreads=4)
+    # alpha = 0 is plain RTN: the loss equals the independent restatement's
+    ref0 = _plain_rtn_loss(X, W)
+    assert abs(losses[0] - ref0) <= 1e-9 * ref0
+    # the choice is the first minimiser, and its scales are that grid point's
+    assert j == int(np.argmin(losses)) and losses[j] == losses.min()
+    m = oracle.act_stats(X)
+    assert np.array_equal(s.view(np.uint16), oracle.scales_alpha(m, j).view(np.uint16))
+    # on data with outlier channels the activation-aware point beats plain RTN
+    assert j > 0 and losses[j] < losses[0]
+
+
+def test_scale_search_power_of_two_invariance():
+    # X * 256: m * 256, so r1, r2, r3 scale by 16, 4, 2 exactly and the normalised
+    # scales are unchanged; Y and Yq scale by 256 and every loss by 2^16 exactly
+    L = synth.make_layer(1, 1, M=1, K=256, N=32, R=16)
+    X = (L.Xcal.numpy().astype(np.float32) / 4).astype(np.float16)
+    X2 = (X.astype(np.float32) * 256).astype(np.float16)
+    assert np.array_equal(X2.astype(np.float64), X.astype(np.float64) * 256)
+    W = L.W.numpy()
+    j1, s1, l1 = oracle.scale_search(X, W)
+    j2, s2, l2 = oracle.scale_search(X2, W)
+    assert j1 == j2 and np.array_equal(s1.view(np.uint16), s2.view(np.uint16))
+    assert np.array_equal(l2, l1 * 65536.0)
