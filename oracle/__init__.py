@@ -62,12 +62,14 @@ def configure(lib):
     lib.awq_oracle_dequant.argtypes = [P, P, P, I64, I64, P]
     lib.awq_oracle_fold_inverse_scale.argtypes = [P, I64, I64, P, P]
     lib.awq_oracle_scales_alpha.argtypes = [P, I64, I, P]
+    lib.awq_oracle_quantize_pack_clip.argtypes = [P, P, P, I64, I64, I64, I, P, P, P, P]
     lib.awq_oracle_scale_search.argtypes = [P, I64, I64, P, I64, P, P, P, I]
     lib.awq_oracle_matmul.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, I, I]
     for f in (lib.awq_oracle_act_stats, lib.awq_oracle_compute_scales,
               lib.awq_oracle_quantize_pack, lib.awq_oracle_quantize_pack_symmetric,
               lib.awq_oracle_dequant, lib.awq_oracle_matmul, lib.awq_oracle_fold_inverse_scale,
-              lib.awq_oracle_scales_alpha, lib.awq_oracle_scale_search):
+              lib.awq_oracle_scales_alpha, lib.awq_oracle_scale_search,
+              lib.awq_oracle_quantize_pack_clip):
         f.restype = ctypes.c_int
     return lib
 
@@ -165,6 +167,30 @@ def quantize_pack(W, s, zero_point: bool = True):
     _check(_load().awq_oracle_quantize_pack(_p(w), _p(sv), K, N, _p(Q), _p(sc), _p(z)),
            "quantize_pack")
     return Q, sc.view(np.float16), z
+
+
+def quantize_pack_clip(W, s, xcal, n_cand: int = 11):
+    """quantize_pack with a searched clipping ratio per (group, column).
+
+    "Awq Quantization", calibration parameters (apply_clip).  Candidates
+    c = 1 - i/20 (i < n_cand); the loss is the group's output error on the
+    calibration rows.  Returns (Q, scales, zeros, ratio_index int32 [K/128, N]).
+    """
+    w = _h(W)
+    sv = _h(s)
+    x = _h(xcal)
+    K, N = w.shape
+    R = x.shape[0]
+    if sv.shape != (K,) or x.shape[1] != K:
+        raise ValueError("s must be [K] and xcal [R, K]")
+    G = max(K // GROUP, 1)
+    Q = np.zeros((max(K // 8, 1), N), dtype=np.int32)
+    sc = np.zeros((G, N), dtype=np.uint16)
+    z = np.zeros((G, max(N // 8, 1)), dtype=np.int32)
+    ri = np.zeros((G, N), dtype=np.int32)
+    _check(_load().awq_oracle_quantize_pack_clip(_p(w), _p(sv), _p(x), R, K, N, int(n_cand), _p(Q),
+                                                 _p(sc), _p(z), _p(ri)), "quantize_pack_clip")
+    return Q, sc.view(np.float16), z, ri
 
 
 def scales_alpha(m, j: int) -> np.ndarray:

@@ -343,6 +343,124 @@ int awq_oracle_quantize_pack(const uint16_t *W, const uint16_t *s, int64_t K, in
 }
 
 /* ---------------------------------------------------------------------------
+ * Weight clipping (next row) -- "Awq Quantization", calibration parameters:
+ * apply_clip = True ("Apply weight clipping"); the page names only the flag.
+ * READINGS:
+ *   candidates  c_i = 1 - i/20, i = 0 .. n_cand-1 (n_cand <= 11: c down to 1/2),
+ *               c_0 = 1 being no clipping
+ *   clipped     per group g and column n, with w' = float(w) * float(s_k):
+ *               hi = c * max w', lo = c * min w' (float products), then step 4 on
+ *               [lo, hi]: r = max(hi - lo, 1e-5f), scale_h = binary16_RNE(r / 15)
+ *               (never 0), z = clamp(rint(-lo / scale_h), 0, 15); every code of the
+ *               group (clipped weights included) q = clamp(rint(w'/scale_h) + z, 0, 15)
+ *   loss        the group's share of the output error on the calibration rows:
+ *               sum_r (sum_{k in g} x'_rk (w_hat_kn - w'_kn))^2 in double, with
+ *               x' = x / s_k in double and w_hat = (q - z) * scale_h
+ *   choice      the first candidate (largest c) with the minimum loss
+ * ratio_index[g * N + n] receives the chosen i.  n_cand = 1 is step 4 exactly.
+ * ------------------------------------------------------------------------ */
+static void group_params(float lo, float hi, uint16_t *sh_out, int32_t *z_out)
+{
+    float r = hi - lo;
+    if (r < 1e-5f)
+        r = 1e-5f;
+    uint16_t sh = f2h(r / 15.0f);
+    if ((sh & 0x7fff) == 0)
+        sh = 1;
+    float zf = nearbyintf(-lo / h2f(sh));
+    if (zf < 0.0f) zf = 0.0f;
+    if (zf > (float)QMAX) zf = (float)QMAX;
+    *sh_out = sh;
+    *z_out = (int32_t)zf;
+}
+
+static int32_t code_of(float w, uint16_t sh, int32_t z)
+{
+    int32_t q = (int32_t)nearbyintf(w / h2f(sh)) + z;
+    if (q < 0) q = 0;
+    if (q > QMAX) q = QMAX;
+    return q;
+}
+
+int awq_oracle_quantize_pack_clip(const uint16_t *W, const uint16_t *s, const uint16_t *xcal, int64_t R,
+                                  int64_t K, int64_t N, int n_cand, int32_t *Q, uint16_t *scales,
+                                  int32_t *zeros, int32_t *ratio_index)
+{
+    if (!W || !s || !xcal || !Q || !scales || !zeros || !ratio_index)
+        return OR_ERR_NULL;
+    if (R < 1 || K < GROUP || K % GROUP != 0 || N < 8 || N % 8 != 0 || n_cand < 1 || n_cand > 11)
+        return OR_ERR_SHAPE;
+    for (int64_t k = 0; k < K; ++k) {
+        float sk = h2f(s[k]);
+        if (!isfinite(sk) || !(sk > 0.0f))
+            return OR_ERR_NONFINITE;
+    }
+    for (int64_t i = 0; i < K * N; ++i)
+        if (!isfinite(h2f(W[i])))
+            return OR_ERR_NONFINITE;
+    int64_t G = K / GROUP;
+    double *xp = (double *)malloc(sizeof(double) * (size_t)(R * GROUP));
+    if (!xp)
+        return OR_ERR_NULL;
+    memset(Q, 0, sizeof(int32_t) * (size_t)((K / 8) * N));
+    memset(zeros, 0, sizeof(int32_t) * (size_t)(G * (N / 8)));
+    for (int64_t g = 0; g < G; ++g) {
+        for (int64_t r = 0; r < R; ++r)
+            for (int64_t kk = 0; kk < GROUP; ++kk) {
+                int64_t k = g * GROUP + kk;
+                xp[r * GROUP + kk] = awq_oracle_half_to_double(xcal[r * K + k]) /
+                                     awq_oracle_half_to_double(s[k]);
+            }
+        for (int64_t n = 0; n < N; ++n) {
+            float wp[GROUP];
+            float mx = -INFINITY, mn = INFINITY;
+            for (int64_t kk = 0; kk < GROUP; ++kk) {
+                int64_t k = g * GROUP + kk;
+                wp[kk] = h2f(W[k * N + n]) * h2f(s[k]);
+                if (wp[kk] > mx) mx = wp[kk];
+                if (wp[kk] < mn) mn = wp[kk];
+            }
+            double best = INFINITY;
+            int best_i = 0;
+            uint16_t best_sh = 0;
+            int32_t best_z = 0;
+            for (int i = 0; i < n_cand; ++i) {
+                float c = 1.0f - (float)i / 20.0f;
+                uint16_t sh;
+                int32_t z;
+                group_params(c * mn, c * mx, &sh, &z);
+                double step = awq_oracle_half_to_double(sh);
+                double e[GROUP];
+                for (int64_t kk = 0; kk < GROUP; ++kk)
+                    e[kk] = (double)(code_of(wp[kk], sh, z) - z) * step - (double)wp[kk];
+                double loss = 0.0;
+                for (int64_t r = 0; r < R; ++r) {
+                    double y = 0.0;
+                    for (int64_t kk = 0; kk < GROUP; ++kk)
+                        y += xp[r * GROUP + kk] * e[kk];
+                    loss += y * y;
+                }
+                if (loss < best) {
+                    best = loss;
+                    best_i = i;
+                    best_sh = sh;
+                    best_z = z;
+                }
+            }
+            ratio_index[g * N + n] = best_i;
+            scales[g * N + n] = best_sh;
+            zeros[g * (N / 8) + n / 8] |= (int32_t)((uint32_t)best_z << (4 * (n % 8)));
+            for (int64_t kk = 0; kk < GROUP; ++kk) {
+                int64_t k = g * GROUP + kk;
+                Q[(k / 8) * N + n] |= (int32_t)((uint32_t)code_of(wp[kk], best_sh, best_z) << (4 * (k % 8)));
+            }
+        }
+    }
+    free(xp);
+    return OR_OK;
+}
+
+/* ---------------------------------------------------------------------------
  * Steps 3-6, symmetric variant -- [P3] "Zero-Point Quantization": with
  * zero_point = False the 4-bit grid has no per-group offset.  The page gives
  * only the flag.

@@ -40,6 +40,8 @@ MUTANTS = {
     "fold multiplies by s": ("f2h(h2f(a[r * K + k]) / h2f(s[k]))", "f2h(h2f(a[r * K + k]) * h2f(s[k]))"),
     "alpha chain: 1/8 power from the square root": ("r3 = sqrt(r2);", "r3 = sqrt(r1);"),
     "scale search keeps the largest loss": ("if (loss < best) {", "if (loss > best) {"),
+    "clip ratio applied to the maximum only": ("group_params(c * mn, c * mx, &sh, &z);", "group_params(mn, c * mx, &sh, &z);"),
+    "clip loss ignores the activations": ("y += xp[r * GROUP + kk] * e[kk];", "y += e[kk];"),
     "missing zeros read as zero": ("if (!zeros)\n        return 8;", "if (!zeros)\n        return 0;"),
 }
 

@@ -621,3 +621,84 @@ def test_scale_search_power_of_two_invariance():
     j2, s2, l2 = oracle.scale_search(X2, W)
     assert j1 == j2 and np.array_equal(s1.view(np.uint16), s2.view(np.uint16))
     assert np.array_equal(l2, l1 * 65536.0)
+
+
+# --------------------------------------------------------------------------
+# weight clipping ("Awq Quantization", calibration parameters: apply_clip)
+# --------------------------------------------------------------------------
+def _group_losses(X16, s, W16, Q, sc, z):
+    """Per (group, column) output error on the calibration rows, from packed outputs (numpy)."""
+    K, N = W16.shape
+    codes, zz = _unpack(Q, z, K, N)
+    wf = W16.astype(np.float32) * s.astype(np.float32)[:, None]
+    wh = (codes - np.repeat(zz, 128, axis=0)) * np.repeat(sc.astype(np.float64), 128, axis=0)
+    e = (wh - wf.astype(np.float64)).reshape(K // 128, 128, N)
+    xp = (X16.astype(np.float64) / s.astype(np.float64)).reshape(X16.shape[0], K // 128, 128)
+    y = np.einsum("rgk,gkn->rgn", xp, e)
+    return (y ** 2).sum(axis=0)                                    # [G, N]
+
+
+def test_clip_without_candidates_is_plain_quantization():
+    L = synth.make_layer(1, 2, M=1, K=384, N=40, R=16)
+    s = oracle.compute_scales(oracle.act_stats(L.Xcal.numpy()))
+    Q, sc, z, ri = oracle.quantize_pack_clip(L.W.numpy(), s, L.Xcal.numpy(), n_cand=1)
+    Qp, scp, zp = oracle.quantize_pack(L.W.numpy(), s)
+    assert np.all(ri == 0)
+    assert np.array_equal(Q, Qp) and np.array_equal(z, zp)
+    assert np.array_equal(sc.view(np.uint16), scp.view(np.uint16))
+
+
+def test_clip_never_raises_a_groups_output_error():
+    L = synth.make_layer(1, 3, M=1, K=512, N=64, R=32)
+    X, W = L.Xcal.numpy(), L.W.numpy()
+    s = oracle.compute_scales(oracle.act_stats(X))
+    Q, sc, z, ri = oracle.quantize_pack_clip(W, s, X)
+    Qp, scp, zp = oracle.quantize_pack(W, s)
+    lc = _group_losses(X, s, W, Q, sc, z)
+    lp = _group_losses(X, s, W, Qp, scp, zp)
+    assert np.all(lc <= lp * (1 + 1e-9))
+    assert np.all((ri == 0) | (lc < lp))          # a clipped group strictly gains
+    assert (ri > 0).any() and (ri == 0).any()
+
+
+def test_clip_drops_an_outlier_that_no_activation_sees():
+    # Every column: weights k/16 (k = 0..15, so the minimum is 0 at any ratio)
+    # plus one weight 1.875 on a channel whose calibration activations are all
+    # zero.  At c = 1/2 the range is [0, 0.9375], the step exactly 1/16, and
+    # every seen weight is represented exactly: loss 0.  At c = 1 (step 1/8)
+    # the odd sixteenths sit on ties and err by 1/16; the ratios in between give
+    # steps on which the sixteenths are not exact.  So c = 1/2 is the only
+    # zero-loss choice and the search must take it.  Columns 8..15 are the
+    # mirror image (maximum 0, outlier -1.875), where only a shrunk lower end
+    # reaches zero loss.
+    rng = np.random.default_rng(44)
+    K, N, R = 128, 16, 8
+    W = (rng.integers(0, 16, (K, N)) / 16.0).astype(np.float16)
+    W[0, :] = 0
+    W[5, :] = np.float16(1.875)
+    W[:, 8:] = -W[:, 8:]
+    X = rng.standard_normal((R, K)).astype(np.float16)
+    X[:, 5] = 0
+    s = np.ones(K, np.float16)
+    Q, sc, z, ri = oracle.quantize_pack_clip(W, s, X)
+    assert np.all(ri == 10)
+    _, zz = _unpack(Q, z, K, N)
+    assert np.all(sc.astype(np.float64) == 1 / 16)
+    assert np.all(zz[:, :8] == 0) and np.all(zz[:, 8:] == 15)
+    assert np.all(_group_losses(X, s, W, Q, sc, z) == 0)
+    Qp, scp, zp = oracle.quantize_pack(W, s)
+    assert np.all(_group_losses(X, s, W, Qp, scp, zp) > 0)
+
+
+def test_clip_keeps_a_lossless_grid_and_rejects_bad_counts():
+    rng = np.random.default_rng(45)
+    W, s, codes = _grid_layer(rng, 256, 24, pow2_s=True)
+    X = rng.standard_normal((8, 256)).astype(np.float16)
+    Q, sc, z, ri = oracle.quantize_pack_clip(W, s, X)
+    assert np.all(ri == 0)                         # loss 0 at c = 1, the first minimiser
+    got, _ = _unpack(Q, z, 256, 24)
+    assert np.array_equal(got, codes)
+    for bad in (0, 12):
+        with pytest.raises(oracle.OracleError) as e:
+            oracle.quantize_pack_clip(W, s, X, n_cand=bad)
+        assert e.value.code == oracle.ERR_SHAPE
