@@ -65,11 +65,20 @@ GEMV_SOURCES = ("weight_only_quantization_quantize_b200/csrc/gemv.cu",
                 "include/awq_b200.h")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source with comments and blank runs removed (what the compiler sees)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
+    """Hash of the decode GEMV's code (comments and layout ignored)."""
     h = hashlib.sha256()
     for rel in GEMV_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(rel.encode() + f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(rel.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -135,20 +144,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def build_layers(awq, nlayers, device, workload=WORKLOAD_ID, zero_point=True):
+def build_layers(awq, nlayers, device, workload=WORKLOAD_ID, zero_point=True, M=1, first=0):
     """Quantize `nlayers` distinct synthetic layers on the GPU (kept packed).
 
     zero_point=False: symmetric weights (no zeros tensor; p["z"] is None)."""
     wl = synth.WORKLOADS[workload]
     layers = []
-    for li in range(nlayers):
+    for li in range(first, first + nlayers):
         projs = []
         for si, (K, N, label) in enumerate(wl.shapes):
-            L = synth.make_layer(workload, li, M=1, K=K, N=N, R=wl.R, device=device, shape_id=si)
+            L = synth.make_layer(workload, li, M=M, K=K, N=N, R=wl.R, device=device, shape_id=si)
             s = awq.compute_scales(awq.act_stats(L.Xcal))
             Q, sc, z = awq.quantize_pack(L.W, s, zero_point=zero_point)
             projs.append(dict(K=K, N=N, label=label, X=L.X, s=s, Q=Q, sc=sc, z=z,
-                              Y=torch.empty(1, N, dtype=torch.float16, device=device)))
+                              Y=torch.empty(M, N, dtype=torch.float16, device=device)))
             del L
         layers.append(projs)
     torch.cuda.synchronize()
@@ -177,6 +186,34 @@ def algorithmic_bytes(M, K, N):
     return weight_bytes(K, N) + 2 * M * K + 2 * K + 2 * M * N
 
 
+def zeroed_workspace(awq, device, shapes, Ms):
+    """One zero-filled workspace large enough for every (M, K, N) call of a run."""
+    need = max(awq.gemm_workspace_size(M, K, N) for M in Ms for K, N in shapes)
+    return torch.zeros(need, dtype=torch.uint8, device=device)
+
+
+def graph_time(step, steps, warmup, stream):
+    """Warm up, capture `steps` calls of step(i) in one CUDA graph, replay once
+    untimed, then time one replay with CUDA events; ms for the whole replay."""
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms
+
+
 def run_ours(args, rank, world, device):
     import weight_only_quantization_quantize_b200 as awq
     awq.lib()
@@ -187,10 +224,11 @@ def run_ours(args, rank, world, device):
     nlayers = max(2, math.ceil(2 * L2 / layer_bytes) + 1)
     layers = build_layers(awq, nlayers, device)
     stream = torch.cuda.current_stream(device)
+    ws = zeroed_workspace(awq, device, [(K, N) for K, N, _ in wl.shapes], [1])
 
     def step(i):
         for p in layers[i % nlayers]:
-            awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"])
+            awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"], workspace=ws)
 
     # warm-up, then capture K steps in one CUDA graph (launch-bound decode loop)
     for i in range(args.warmup):
@@ -233,7 +271,7 @@ def run_ours(args, rank, world, device):
     traffic = stored_traffic("gemv_decode_7b")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "peak_source": peak_src,
+                "traffic": traffic, "peak_source": f"{peak_src} HBM copy bandwidth",
                 "kernel": "gemv_kernel",
                 "bytes_per_launch_avg": round(alg_step / 4)}
 
@@ -242,12 +280,15 @@ def run_ours(args, rank, world, device):
 
     extra = {}
     if not args.quick and rank == 0:
-        extra["prefill_7b_m4096"] = run_prefill(awq, device, peaks)
-        extra["quantize_7b_layer"] = run_quantize(awq, device, layers, peaks)
-        extra["small_batch_13b_m48"] = run_small_batch(awq, device, peaks)
-        extra["quantize_7b_layer_symmetric"] = run_quantize(awq, device, layers, peaks, zero_point=False)
-        extra["decode_7b_symmetric"] = run_decode_symmetric(awq, device, peaks, nlayers)
-        extra["decode_7b_prescaled"] = run_decode_symmetric(awq, device, peaks, nlayers, prescaled=True)
+        del layers
+        torch.cuda.empty_cache()
+        extra.update(run_config_sweep(awq, device, peaks, peak_src))
+        qlayers = build_layers(awq, 1, device)
+        extra["quantize_7b_layer"] = run_quantize(awq, device, qlayers, peaks)
+        extra["quantize_7b_layer_symmetric"] = run_quantize(awq, device, qlayers, peaks, zero_point=False)
+        del qlayers
+        extra["decode_7b_symmetric"] = run_decode_variant(awq, device, peaks, nlayers)
+        extra["decode_7b_prescaled"] = run_decode_variant(awq, device, peaks, nlayers, prescaled=True)
 
     cpu = run_cpu_baseline(rank, world) if rank == 0 else None
     return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, launches=launches,
@@ -257,7 +298,8 @@ def run_ours(args, rank, world, device):
 def run_e2e(awq, layers, args, device):
     """The decode step through the public API with host buffers: every step
     copies that layer's four activation rows from pinned host memory (one
-    copy), runs the four GEMVs and reads the four outputs back (one copy)."""
+    copy), runs the four projections (QuantLinear layers, eager) and reads the
+    four outputs back (one copy)."""
     stream = torch.cuda.current_stream(device)
     nl = len(layers)
     ks = [p["K"] for p in layers[0]]
@@ -273,14 +315,15 @@ def run_e2e(awq, layers, args, device):
             hx[li][xo[pi]:xo[pi + 1]].copy_(p["X"].view(-1).cpu())
     xv = [[dx[li][xo[pi]:xo[pi + 1]].view(1, -1) for pi in range(len(ks))] for li in range(nl)]
     yv = [[dy[li][yo[pi]:yo[pi + 1]].view(1, -1) for pi in range(len(ns))] for li in range(nl)]
+    lin = [[awq.QuantLinear(p["Q"], p["sc"], p["z"], p["s"]) for p in layer] for layer in layers]
     h2d = 2 * int(xo[-1])
     d2h = 2 * int(yo[-1])
 
     def step(i):
         li = i % nl
         dx[li].copy_(hx[li], non_blocking=True)
-        for pi, p in enumerate(layers[li]):
-            awq.w4a16_gemv(xv[li][pi], p["s"], p["Q"], p["sc"], p["z"], out=yv[li][pi])
+        for pi, f in enumerate(lin[li]):
+            f(xv[li][pi], out=yv[li][pi])
         hy[li].copy_(dy[li], non_blocking=True)
 
     for i in range(args.warmup):
@@ -297,90 +340,78 @@ def run_e2e(awq, layers, args, device):
     return {"value": round(wb * args.steps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4),
-            "path": "python binding -> C ABI, eager; one H2D copy of the step's 4 activation rows, one D2H copy of its 4 outputs"}
+            "path": "QuantLinear (python binding -> C ABI), eager; one H2D copy of the step's 4 "
+                    "activation rows, one D2H copy of its 4 outputs"}
 
 
 def flush_l2(buf):
     buf.add_(1)
 
 
-def run_prefill(awq, device, peaks, M=4096, reps=5):
-    """7B prefill GEMMs (tcgen05 path), TFLOP/s over the four shapes."""
-    wl = synth.WORKLOADS[4]
-    projs = []
-    for si, (K, N, label) in enumerate(wl.shapes):
-        L = synth.make_layer(4, 0, M=M, K=K, N=N, R=wl.R, device=device, shape_id=si)
-        s = awq.compute_scales(awq.act_stats(L.Xcal))
-        Q, sc, z = awq.quantize_pack(L.W, s)
-        ws = torch.empty(awq.gemm_workspace_size(M, K, N), dtype=torch.uint8, device=device)
-        projs.append(dict(K=K, N=N, X=L.X, s=s, Q=Q, sc=sc, z=z, ws=ws,
-                          Y=torch.empty(M, N, dtype=torch.float16, device=device)))
-        del L
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-
-    def step():
-        for p in projs:
-            awq.w4a16_gemm(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"], workspace=p["ws"])
-
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(reps):
-        flush_l2(flush)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
-    flops = sum(2 * M * p["K"] * p["N"] for p in projs)
-    tf = flops / (ms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    return {"M": M, "ms_per_layer": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak,
-            "frac": round(tf / peak, 4), "includes": "X/s pre-pass + tcgen05 GEMM, 4 shapes",
-            "l2": "256 MB buffer rewritten before each timed layer"}
+def _sweep_entry(kind, M, wl, ms_per_pass, passes_bytes, flops, peaks, peak_src, layers_note):
+    """One sweep key: weight GB/s for the HBM-bound token counts, TFLOP/s (and
+    GB/s) for the tensor-bound ones, each as a fraction of the named peak."""
+    gbs = passes_bytes / (ms_per_pass * 1e-3) / 1e9
+    tf = flops / (ms_per_pass * 1e-3) / 1e12
+    e = {"M": M, "shapes": [list(x[:2]) for x in wl.shapes], "ms_per_pass": round(ms_per_pass, 5),
+         "weight_gbs": round(gbs, 1), "tflops": round(tf, 1), "layers": layers_note}
+    if kind == "hbm":
+        e.update(bound="hbm", frac=round(gbs / peaks["hbm_gbs"], 4), peak=peaks["hbm_gbs"],
+                 peak_name=f"{peak_src} HBM copy bandwidth (GB/s)")
+    else:
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        e.update(bound="tensor", frac=round(tf / peak, 4), peak=peak,
+                 peak_name=f"{peak_src} dense bf16 burst (TFLOP/s; fp16 runs at the bf16 rate); "
+                           "each pass is a few ms timed alone")
+    return e
 
 
-def run_small_batch(awq, device, peaks, M=48, reps=10):
-    """13B small-batch GEMMs (register-fed tensor cores), weight GB/s."""
-    wl = synth.WORKLOADS[3]
-    projs = []
-    for si, (K, N, label) in enumerate(wl.shapes):
-        L = synth.make_layer(3, 0, M=M, K=K, N=N, R=wl.R, device=device, shape_id=si)
-        s = awq.compute_scales(awq.act_stats(L.Xcal))
-        Q, sc, z = awq.quantize_pack(L.W, s)
-        ws = torch.empty(awq.gemm_workspace_size(M, K, N), dtype=torch.uint8, device=device)
-        projs.append(dict(K=K, N=N, X=L.X, s=s, Q=Q, sc=sc, z=z, ws=ws,
-                          Y=torch.empty(M, N, dtype=torch.float16, device=device)))
-        del L
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+def run_sweep(awq, device, peaks, peak_src, wid, Ms, reps, kinds):
+    """Time `reps` passes over distinct layers of workload `wid` for each token
+    count in Ms, each captured in one CUDA graph (layers rotate so the weights
+    come from HBM).  The layers are quantized once, with activations for the
+    largest M; smaller M use the leading rows."""
+    wl = synth.WORKLOADS[wid]
+    L2 = torch.cuda.get_device_properties(device).L2_cache_size
+    layer_bytes = sum(weight_bytes(K, N) for K, N, _ in wl.shapes)
+    nlayers = wl.layers if wl.layers > 1 else max(2, math.ceil(2 * L2 / layer_bytes) + 1)
+    Mmax = max(Ms)
+    layers = build_layers(awq, nlayers, device, workload=wid, M=Mmax)
+    ws = zeroed_workspace(awq, device, [(K, N) for K, N, _ in wl.shapes], Ms)
+    stream = torch.cuda.current_stream(device)
+    note = (f"{nlayers} distinct layers, each pass one layer's 4 projections" if wl.layers > 1 else
+            f"{nlayers} distinct layers rotated ({nlayers * layer_bytes / 1e6:.0f} MB packed > 2 x L2)")
+    out = {}
+    for M, kind in zip(Ms, kinds):
+        views = [[(p, p["X"][:M], p["Y"][:M]) for p in layer] for layer in layers]
 
-    def step():
-        for p in projs:
-            awq.w4a16_gemm(p["X"], p["s"], p["Q"], p["sc"], p["z"], out=p["Y"], workspace=p["ws"])
+        def step(i):
+            for p, X, Y in views[i % nlayers]:
+                awq.w4a16_gemm(X, p["s"], p["Q"], p["sc"], p["z"], out=Y, workspace=ws)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(reps):
-        flush_l2(flush)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
-    wb = sum(weight_bytes(p["K"], p["N"]) for p in projs)
-    gbs = wb / (ms * 1e-3) / 1e9
-    return {"M": M, "ms_per_layer": round(ms, 4), "weight_gbs": round(gbs, 1),
-            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "includes": "X/s pre-pass + 4 GEMMs"}
+        steps = reps * nlayers if wl.layers > 1 else max(reps, nlayers)
+        ms = graph_time(step, steps, 3, stream) / steps
+        flops = sum(2 * M * K * N for K, N, _ in wl.shapes)
+        out[M] = _sweep_entry(kind, M, wl, ms, layer_bytes, flops, peaks, peak_src, note)
+    del layers, ws
+    torch.cuda.empty_cache()
+    return out
 
 
-def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5, prescaled=False):
+def run_config_sweep(awq, device, peaks, peak_src):
+    """Every workload and token count of the benchmark configuration list."""
+    out = {}
+    out["single_layer_1024_m1"] = run_sweep(awq, device, peaks, peak_src, 1, [1], 200, ["hbm"])[1]
+    r = run_sweep(awq, device, peaks, peak_src, 3, [8, 16, 32, 48], 20, ["hbm"] * 4)
+    out.update({f"small_batch_13b_m{M}": e for M, e in r.items()})
+    r = run_sweep(awq, device, peaks, peak_src, 4, [512, 2048, 4096], 5, ["tensor"] * 3)
+    out.update({f"prefill_7b_m{M}": e for M, e in r.items()})
+    r = run_sweep(awq, device, peaks, peak_src, 5, [1, 32, 256], 2, ["hbm", "hbm", "tensor"])
+    out.update({f"stack_70b_m{M}": e for M, e in r.items()})
+    return out
+
+
+def run_decode_variant(awq, device, peaks, nlayers, steps=200, warmup=5, prescaled=False):
     """A decode-step variant, timed like the headline.
 
     prescaled=False: symmetric weights (zeros = NULL); algorithmic bytes 0.5 B
@@ -394,30 +425,17 @@ def run_decode_symmetric(awq, device, peaks, nlayers, steps=200, warmup=5, presc
             for p in lp:
                 p["X"] = awq.fold_inverse_scale(p["X"], p["s"])
         torch.cuda.synchronize()
+    ws = zeroed_workspace(awq, device, [(K, N) for K, N, _ in wl.shapes], [1])
 
     def step(i):
         for p in layers[i % nlayers]:
             if prescaled:
-                awq.w4a16_gemv(p["X"], None, p["Q"], p["sc"], p["z"], out=p["Y"])
+                awq.w4a16_gemv(p["X"], None, p["Q"], p["sc"], p["z"], out=p["Y"], workspace=ws)
             else:
-                awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], None, out=p["Y"])
+                awq.w4a16_gemv(p["X"], p["s"], p["Q"], p["sc"], None, out=p["Y"], workspace=ws)
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i in range(steps):
-            step(i)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    del g, layers
+    ms = graph_time(step, steps, warmup, torch.cuda.current_stream(device))
+    del layers
     per_weight = BYTES_PER_WEIGHT if prescaled else 0.5 + 2 / 128
     wbytes = sum(K * N * per_weight for K, N, _ in wl.shapes)
     gbs = wbytes * steps / (ms * 1e-3) / 1e9

@@ -30,6 +30,9 @@
  *     dev_status is not NULL; the first error wins, the library never clears
  *     it: the caller zeroes it and reads it after synchronizing the stream.
  *   - Outputs must not alias inputs.
+ *   - The library keeps per-device state (device checks, kernel attributes,
+ *     encoded tensor maps, the no-allocation scratch address): do not use it
+ *     on a device after cudaDeviceReset in the same process.
  *
  * Data layout (K input channels, N output channels, G = K/128 groups)
  *   W       binary16 [K, N]     Y = X W
@@ -64,7 +67,9 @@ extern "C" {
 #define AWQ_MAX_K 262144
 #define AWQ_MAX_N 1048576
 #define AWQ_MAX_M 1048576
-#define AWQ_ABI_VERSION 3  /* 2: symmetric weights; 3: 1/s folded upstream */
+#define AWQ_ABI_VERSION 4  /* 2: symmetric weights; 3: 1/s folded upstream;
+                               4: every matmul takes a zero-filled workspace;
+                               scale search over alpha; weight clipping */
 
 typedef enum {
     AWQ_OK = 0,
@@ -152,6 +157,38 @@ AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16
                                          int32_t *dev_status, awq_stream_t stream);
 
 /*
+ * Fold, quantize and pack with weight clipping -- "Awq Quantization",
+ * calibration parameters: apply_clip ("Apply weight clipping"); the page names
+ * only the flag.  This library reads it, per group g (rows 128g..128g+127)
+ * and column n with w' = float(w) * float(s_k), as:
+ *   candidates  c_i = 1 - i/20, i = 0 .. n_cand-1 (1 <= n_cand <= 11, down to
+ *               c = 1/2; c_0 = 1 is no clipping)
+ *   clipped     lo = c * min w', hi = c * max w' (float); step and zero point
+ *               from [lo, hi] as in awq_quantize_pack (r = max(hi - lo, 1e-5f),
+ *               scale_h = binary16_RNE(r / 15), z = clamp(rint(-lo / scale_h),
+ *               0, 15)); every weight of the group coded on that grid,
+ *               q = clamp(rint(w' / scale_h) + z, 0, 15)
+ *   loss        sum over the R calibration rows of
+ *               (sum_{k in g} (xcal[r,k] / s_k) ((q - z) scale_h - w'))^2
+ *               (float arithmetic)
+ *   choice      the first candidate (largest c) with the minimum loss.
+ * With n_cand = 1 the outputs equal awq_quantize_pack's bit for bit.  The
+ * step, zero point and codes of a chosen candidate are bit-exact functions of
+ * W, s and that candidate; the choice itself rests on float losses, so it can
+ * differ from an exact (double) evaluation only between candidates whose
+ * losses agree to float rounding.
+ *   W binary16 [K, N], s binary16 [K] (> 0), xcal binary16 [R, K]
+ *   (1 <= R <= AWQ_MAX_CALIB_ROWS), K % 128 == 0, N % 8 == 0
+ *   Q, scales, zeros as for awq_quantize_pack (outputs); ratio_index int32
+ *   [K/128, N] receives the chosen i (may be NULL)
+ * Device errors: AWQ_ERR_NONFINITE for NaN/Inf in W, s or xcal, or s <= 0.
+ */
+AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s, const uint16_t *xcal,
+                                            int64_t R, int64_t K, int64_t N, int32_t n_cand, int32_t *Q,
+                                            uint16_t *scales, int32_t *zeros, int32_t *ratio_index,
+                                            int32_t *dev_status, awq_stream_t stream);
+
+/*
  * Fused-dequantization matmul -- lansai explainer, "AWQ 的四步链路"
  * (Y = (X/s)(sW)); "Awq Quantization", "WQLinear Kernel Variants" (GEMV for
  * batch size 1, GEMM for batches).
@@ -165,7 +202,8 @@ AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16
  * awq_w4a16_gemv is the M = 1 (single-token decode) entry point:
  *   X binary16 [1, K], Y binary16 [1, N].
  * awq_w4a16_gemm takes any 1 <= M <= AWQ_MAX_M and picks its tile path
- * internally: the decode GEMV for M <= 2, register-fed tensor cores for
+ * internally: the decode GEMV for M <= 2 (persistent, one CTA per SM, split
+ * tiles finished by the last-arriving worker), register-fed tensor cores for
  * 3 <= M < 40, tcgen05/TMEM for M >= 40 (small batch from 40, prefill from 64).
  *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack;
  *   zeros = NULL for weights from awq_quantize_pack_symmetric (zero point 8).
@@ -173,17 +211,22 @@ AWQ_API awq_status_t awq_quantize_pack_symmetric(const uint16_t *W, const uint16
  *   produced X, e.g. by awq_fold_inverse_scale): X is then used as it is, and
  *   with X = awq_fold_inverse_scale(X, s) the result equals, bit for bit,
  *   the call with the original X and s.
- * Workspace: caller-owned device memory of at least *_workspace_size() bytes
- * (may be NULL when that size is 0); it holds X / s and is overwritten.
+ * Workspace: caller-owned device memory of at least *_workspace_size() bytes,
+ * never NULL.  It must be zero-filled (e.g. cudaMemsetAsync) before its first
+ * use: its first 32 KB hold arrival counters that a call expects at zero and
+ * leaves at zero when it completes without a device error.  The rest holds
+ * X / s and partial sums and is overwritten.  Calls on one stream may share a
+ * workspace; calls that can run at the same time need separate ones.  After a
+ * device error (AWQ_ERR_DEVICE_TIMEOUT) zero the workspace again.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
  * (Y is then unspecified).
  * Stream ordering: these kernels use programmatic dependent launch, so a call
- * may start while the previous kernel on the stream is still finishing.  X is
- * read only after that kernel has completed.  Q, scales and zeros are treated
- * as layer state and may be read before it completes: they must not be
- * written by a kernel that triggers programmatic dependent launch early.
- * Ordinary kernels, copies and awq_quantize_pack complete before any
- * dependent starts, so writing the weights with them is safe.
+ * may start while the previous kernel on the stream is still finishing.  X and
+ * the workspace are touched only after that kernel has completed.  Q, scales
+ * and zeros are treated as layer state and may be read before it completes:
+ * they must not be written by a kernel that triggers programmatic dependent
+ * launch early.  Ordinary kernels, copies and awq_quantize_pack complete before
+ * any dependent starts, so writing the weights with them is safe.
  */
 /*
  * Fold 1/s upstream -- lansai explainer, "AWQ 的四步链路": Y = XW = (X/s)(sW),
@@ -213,6 +256,49 @@ AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const 
                             int32_t *dev_status, awq_stream_t stream);
 
 /*
+ * Scales of one grid point of the scale search (below): alpha = j/8,
+ * 0 <= j <= 8, by the same fixed chain of IEEE double operations,
+ *   s = binary16_RNE(t / sqrt(max t * min t)),  t = m^(j/8)
+ * (j = 4 gives awq_compute_scales bit for bit, j = 0 gives s = 1).
+ *   m float [K] (K >= 1); s binary16 [K] (output)
+ * Device errors: AWQ_ERR_NONFINITE if some m_k is NaN/Inf/negative.
+ */
+AWQ_API awq_status_t awq_scales_alpha(const float *m, int64_t K, int32_t j, uint16_t *s,
+                                      int32_t *dev_status, awq_stream_t stream);
+
+/*
+ * Scale search over alpha -- "Awq Quantization", "How AWQ Works" (s is chosen
+ * to make L(s) = ||Q(W*s)(s^-1*X) - W*X|| small); lansai explainer, "AWQ 的四步
+ * 链路", row "搜索缩放" (try channel scalings, keep the one with the smallest
+ * reconstruction error).  The pages give neither the family nor the grid;
+ * this library reads them as:
+ *   family  s(alpha) = m^alpha normalised as in awq_compute_scales (whose scale
+ *           is the alpha = 1/2 point), m = awq_act_stats(xcal)
+ *   grid    alpha = j/8, j = 0..8, m^alpha by one fixed chain of IEEE double
+ *           operations: u = max(m, 1e-8), r1 = sqrt(u), r2 = sqrt(r1),
+ *           r3 = sqrt(r2); t = u for j = 8, else the product of r1, r2, r3
+ *           selected by the bits 4, 2, 1 of j, in that order;
+ *           s = binary16_RNE(t / sqrt(max t * min t))
+ *   loss    losses[j] = sum over the R calibration rows and N outputs of
+ *           (Yq - Y)^2 (double), Yq = awq_w4a16_gemm(xcal, s(j), awq_quantize_pack(W, s(j)))
+ *           and Y = xcal W (tensor cores, float accumulation)
+ *   choice  *j_best = the smallest j with the minimum loss; s_best = s(j_best),
+ *           bit for bit the scale of that grid point.
+ *   xcal  binary16 [R, K], 1 <= R <= AWQ_MAX_CALIB_ROWS; W binary16 [K, N],
+ *         K % 128 == 0, N % 8 == 0
+ *   losses double [9], s_best binary16 [K], j_best int32 [1] (device outputs)
+ *   workspace  at least awq_scale_search_workspace_size(R, K, N) bytes,
+ *         zero-filled before its first use (it embeds a matmul workspace)
+ * Device errors: AWQ_ERR_NONFINITE for NaN/Inf in xcal or W (the outputs are
+ * then unspecified); AWQ_ERR_DEVICE_TIMEOUT as for the matmul.
+ */
+AWQ_API size_t awq_scale_search_workspace_size(int64_t R, int64_t K, int64_t N);
+AWQ_API awq_status_t awq_scale_search(const uint16_t *xcal, int64_t R, int64_t K, const uint16_t *W,
+                                      int64_t N, double *losses, uint16_t *s_best, int32_t *j_best,
+                                      void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                      awq_stream_t stream);
+
+/*
  * awq_w4a16_gemm_noalloc -- awq_w4a16_gemm for callers that cannot hand the
  * library a workspace.  No counterpart in the AWQ paper or pages: this is an
  * integration entry point of this library only.
@@ -229,16 +315,19 @@ AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const 
  *
  * Arguments, layouts, tolerance and errors are those of awq_w4a16_gemm, minus
  * the workspace.  Limit: awq_w4a16_gemm_workspace_size(M, K, N) must not exceed
- * AWQ_NOALLOC_SCRATCH_BYTES (2 * M * K bytes for M > 1, i.e. M * K <= 2 Mi
- * elements); larger problems return AWQ_ERR_WORKSPACE before anything runs.
+ * AWQ_NOALLOC_SCRATCH_BYTES (32 KB of counters + 2 * M * K bytes of X / s, plus
+ * 768 KB per token for M <= 2; for example M * K <= 2 Mi elements at M >= 3);
+ * larger problems return AWQ_ERR_WORKSPACE before anything runs.
  * Set-up: the first call on each device (with that device current) looks up
  * the scratch array's device address; make that first call before any stream
  * capture begins.
  * Sharing: every call on a device uses the same scratch array, which keeps the
- * last call's contents (nothing in it needs to start at zero: each call writes
- * the part it reads).  Calls whose executions overlap on the GPU (different
- * streams without ordering between them) race on the scratch array and give
- * undefined results; order them on one stream or with events.
+ * last call's contents.  Its counter block starts at zero (the array is
+ * zero-initialised when the library is loaded) and every call that completes
+ * without a device error leaves it at zero; the rest is written before it is
+ * read.  Calls whose executions overlap on the GPU (different streams without
+ * ordering between them) race on the scratch array and give undefined
+ * results; order them on one stream or with events.
  */
 #define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 AWQ_API awq_status_t awq_w4a16_gemm_noalloc(const uint16_t *X, const uint16_t *s, const int32_t *Q,

@@ -52,18 +52,24 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.awq_abi_version() == 3
+    assert L.awq_abi_version() == 4 == awq.ABI_VERSION
     for code, name in awq.STATUS.items():
         assert awq.status_string(code).startswith(name)
     assert awq.status_string(99) == "AWQ_ERR_UNKNOWN"
 
 
 def test_workspace_sizes(L):
-    assert L.awq_w4a16_gemv_workspace_size(4096, 4096) == 0
-    assert L.awq_w4a16_gemm_workspace_size(1, 4096, 4096) == 0
-    assert L.awq_w4a16_gemm_workspace_size(48, 5120, 5120) >= 2 * 48 * 5120
-    assert L.awq_w4a16_gemm_workspace_size(4096, 14336, 4096) >= 2 * 4096 * 14336
+    # every matmul takes a workspace: 32 KB of arrival counters first, then
+    # X / s (2 M K bytes), then (M <= 2) the decode GEMV's partial sums
+    counters = 32 * 1024
+    g1 = L.awq_w4a16_gemv_workspace_size(4096, 4096)
+    assert g1 == L.awq_w4a16_gemm_workspace_size(1, 4096, 4096)
+    assert g1 >= counters + 2 * 4096
+    assert L.awq_w4a16_gemm_workspace_size(2, 4096, 4096) > g1
+    assert L.awq_w4a16_gemm_workspace_size(48, 5120, 5120) >= counters + 2 * 48 * 5120
+    assert L.awq_w4a16_gemm_workspace_size(4096, 14336, 4096) >= counters + 2 * 4096 * 14336
     assert L.awq_w4a16_gemm_workspace_size(4, 100, 4096) == 0          # invalid shape
+    assert L.awq_w4a16_gemv_workspace_size(4096, 4097) == 0            # invalid shape
 
 
 def gemm(L, X=A, s=A, Q=A, sc=A, z=A, M=64, K=4096, N=4096, Y=A, ws=A, wsb=1 << 40, st=None):
@@ -127,3 +133,30 @@ def test_quantize_and_stats_validation(L):
     cs = L.awq_compute_scales
     assert cs(P(A), 0, P(A), None, None) == awq.ERR_SHAPE
     assert cs(P(A), 16, P(0), None, None) == awq.ERR_NULL
+
+
+def test_scale_search_validation(L):
+    ss = L.awq_scale_search
+    ws = L.awq_scale_search_workspace_size(256, 4096, 4096)
+    assert ws > 2 * 4096 * 4096 + 4 * 256 * 4096             # holds W transposed and X W in float
+    assert L.awq_scale_search_workspace_size(0, 4096, 4096) == 0     # empty calibration
+    assert L.awq_scale_search_workspace_size(9000, 4096, 4096) == 0  # above the exact-sum limit
+    assert L.awq_scale_search_workspace_size(256, 100, 4096) == 0
+
+    def call(x=A, R=256, K=4096, w=A, N=4096, lo=A, sb=A, jb=A, wsp=A, wsb=ws, st=None):
+        return ss(P(x), R, K, P(w), N, P(lo), P(sb), P(jb), P(wsp), wsb, P(st), None)
+    assert call(x=0) == awq.ERR_NULL
+    assert call(jb=0) == awq.ERR_NULL
+    assert call(R=0) == awq.ERR_SHAPE
+    assert call(K=200) == awq.ERR_SHAPE
+    assert call(N=20) == awq.ERR_SHAPE
+    assert call(sb=MIS) == awq.ERR_ALIGN
+    assert call(jb=A + 2) == awq.ERR_ALIGN
+    assert call(wsp=0) == awq.ERR_WORKSPACE
+    assert call(wsb=ws - 1) == awq.ERR_WORKSPACE
+    sa = L.awq_scales_alpha
+    assert sa(P(0), 16, 4, P(A), None, None) == awq.ERR_NULL
+    assert sa(P(A), 16, 9, P(A), None, None) == awq.ERR_SHAPE
+    assert sa(P(A), 16, -1, P(A), None, None) == awq.ERR_SHAPE
+    assert sa(P(A), 0, 4, P(A), None, None) == awq.ERR_SHAPE
+    assert sa(P(A), 16, 4, P(MIS), None, None) == awq.ERR_ALIGN

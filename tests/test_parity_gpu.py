@@ -243,3 +243,46 @@ def test_full_size_7b_prefill(shape_id, M):
 @pytest.mark.parametrize("shape_id,M", [(0, 1), (1, 32), (3, 256), (2, 1)])
 def test_full_size_70b_layer(shape_id, M):
     _check_full(5, shape_id, M, 96, 400 + shape_id)
+
+
+# ------------------------------------------------------------------ stream ordering and workspace state
+def test_quantize_then_matmul_on_one_stream_without_sync():
+    # The matmul fetches its packed weights before it waits on the previous
+    # kernel of the stream (programmatic dependent launch).  The quantizer
+    # triggers its dependents only when it completes, so a matmul issued right
+    # behind it on the same stream, with no synchronization in between, must
+    # read the freshly written weights.
+    L = synth.make_layer(15, 0, M=1, K=4096, N=6144, R=64)
+    sr = oracle.compute_scales(oracle.act_stats(h(L.Xcal)))
+    Qr, scr, zr = oracle.quantize_pack(h(L.W), sr)
+    Yref = oracle.matmul(h(L.X), sr, Qr, scr, zr, precision=64, nthreads=16)
+    Wd, sd, Xd = dev(L.W), dev(torch.from_numpy(sr)), dev(L.X)
+    Q = torch.zeros(4096 // 8, 6144, dtype=torch.int32, device="cuda")
+    sc = torch.zeros(32, 6144, dtype=torch.float16, device="cuda")
+    z = torch.zeros(32, 768, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    for M in (1, 2, 16, 48, 128):
+        X = dev(synth.activations(M, 4096, 17 + M, L.outliers))
+        Q.zero_()
+        awq.quantize_pack(Wd, sd, out=(Q, sc, z))            # no sync after this
+        Y = awq.w4a16_gemm(X, sd, Q, sc, z)
+        Yr = oracle.matmul(h(X), sr, Qr, scr, zr, precision=64, nthreads=16)
+        assert_y_close(Y.cpu().numpy(), Yr, f"M={M} right after quantize_pack")
+    Q.zero_()
+    awq.quantize_pack(Wd, sd, out=(Q, sc, z))
+    assert_y_close(awq.w4a16_gemv(Xd, sd, Q, sc, z).cpu().numpy(), Yref, "gemv right after quantize_pack")
+
+
+def test_workspace_counters_return_to_zero():
+    # The decode GEMV counts arrivals on split tiles in the first 32 KB of the
+    # workspace; every call must leave them at zero for the next one.
+    ws = torch.zeros(awq.gemm_workspace_size(2, 14336, 28672), dtype=torch.uint8, device="cuda")
+    for (K, N, M) in [(4096, 6144, 1), (14336, 4096, 2), (1152, 1032, 1), (128, 8, 2), (4096, 28672, 1)]:
+        L = synth.make_layer(16, K + N, M=M, K=K, N=N, R=64, device="cuda")
+        s = awq.compute_scales(awq.act_stats(L.Xcal))
+        Q, sc, z = awq.quantize_pack(L.W, s)
+        Y1 = awq.w4a16_gemm(L.X, s, Q, sc, z, workspace=ws)
+        Y2 = awq.w4a16_gemm(L.X, s, Q, sc, z, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:32 * 1024].view(torch.int32).abs().sum().item()) == 0, (K, N, M)
+        assert torch.equal(Y1, Y2)

@@ -8,13 +8,12 @@ an entry point that needs no workspace: it stages X / s in a fixed scratch
 array inside the library's device image instead.
 
 These tests call it through the C ABI (ctypes, no Python wrapper) and compare
-its output with the workspace-taking awq_w4a16_gemm on the same inputs, for
-several calls in a row (the scratch array is shared by every call and keeps the
-previous call's contents).  The file is named so that pytest collects it last.
+its output with the workspace-taking awq_w4a16_gemm on the same inputs, bit for
+bit (both run the same kernels), for several calls in a row (the scratch array
+is shared by every call and keeps the previous call's contents).  The file is named so that pytest collects it last.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -29,8 +28,9 @@ def _p(t):
 
 
 def test_noalloc_refuses_problems_larger_than_its_scratch():
-    # 2 * M * K bytes of X / s staging must fit the fixed array; refused before
-    # any device work, so this runs without a GPU (the pointers are never used).
+    # the call's workspace (counters + 2 * M * K bytes of X / s staging) must fit
+    # the fixed array; refused before any device work, so this runs without a
+    # GPU (the pointers are never used).
     L = awq.lib()
     A = P(0x7F0000000000)
     M, K = 4096, 4096
@@ -44,13 +44,6 @@ def _layer(M, K, N, seed):
     s = awq.compute_scales(awq.act_stats(Lr.Xcal))
     Q, sc, z = awq.quantize_pack(Lr.W, s)
     return Lr.X, s, Q, sc, z
-
-
-def _close(y, ref):
-    y = y.double().cpu().numpy()
-    ref = ref.double().cpu().numpy()
-    assert np.abs(y - ref).max() <= 1e-2 * np.abs(ref).max()
-    assert np.linalg.norm(y - ref) <= 5e-3 * np.linalg.norm(ref)
 
 
 @pytest.mark.gpu
@@ -76,4 +69,5 @@ def test_noalloc_matches_gemm_on_consecutive_calls():
         torch.cuda.synchronize()
         assert int(st.item()) == awq.OK
         assert torch.isfinite(Y).all()
-        _close(Y, ref)
+        # same kernels on the same inputs: the result is the same bits
+        assert torch.equal(Y, ref), f"M={M} K={K} N={N}"

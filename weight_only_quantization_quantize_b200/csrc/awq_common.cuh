@@ -21,7 +21,16 @@ constexpr int kGroup = 128;
 // caller then skips its remaining work but still reaches every block- and
 // cluster-wide barrier, so the context survives and the host can read the
 // status word.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+// AWQ_WAIT_LIMIT_NS exists for the test build that checks the timeout path
+// (a wait that does not complete at once then runs out); the library itself
+// is always built with the default.
+#ifndef AWQ_WAIT_LIMIT_NS
+#define AWQ_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = AWQ_WAIT_LIMIT_NS;  // 1 s
+// After a wait has run out, a kernel still lets the copies it issued land
+// before it exits; those waits use their own limit.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s
 
 __device__ __forceinline__ void report(int32_t *status, int code)
 {
@@ -76,16 +85,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return done != 0;
 }
 
-// Wait for the phase with the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// Wait for the phase with the given parity to complete; false once
+// `limit_ns` has passed.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(a, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs) return false;
+        if ((i & 255u) == 0 && globaltimer() - t0 > limit_ns) return false;
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -104,6 +119,20 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int x, int y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
+// Prefetch the L2 line holding `p`.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch
@@ -302,6 +331,23 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(remote_addr),
                  "f"(v), "r"(remote_bar)
                  : "memory");
+}
+
+// ---------------------------------------------------------------- binary16 rounding
+// Round a positive finite double to the nearest binary16, ties to even, in a
+// single rounding (IEEE 754 binary16: quantum 2^(e-10) in the binade
+// [2^e, 2^(e+1)), never finer than the subnormal quantum 2^-24).
+__device__ __forceinline__ uint16_t double_to_half_rn(double x)
+{
+    if (!(x < 65520.0)) return 0x7C00;  // rounds to +inf (x >= 65520)
+    if (x == 0.0) return 0;
+    const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
+    int e = static_cast<int>((b >> 52) & 0x7FF) - 1023;  // x normal in double here
+    int q = e - 10;
+    if (q < -24) q = -24;
+    const double inv_quantum = __longlong_as_double(static_cast<long long>(1023 - q) << 52);
+    const double n = rint(__dmul_rn(x, inv_quantum));  // exact scaling, then RNE
+    return static_cast<uint16_t>(((q + 24) << 10) + static_cast<int>(n));
 }
 
 // ---------------------------------------------------------------- 4-bit unpack

@@ -19,22 +19,23 @@ cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K,
 cudaError_t launch_fold_inverse_scale(const __half *a, int64_t rows, int K, const __half *s,
                                       __half *out, int32_t *status, int num_sms, cudaStream_t st);
 
-// gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group
+// gemv.cu -- M <= 2: decode GEMV, persistent stream-K over (tile, group)
+// units, zero point and step applied once per group
+constexpr int kGemvMaxCtas = 256;  // upper bound of the persistent grid
 struct GemvPlan {
-    int splits;       // CTAs per cluster along K
+    int ctas;         // persistent CTAs (at most one per SM)
+    int stages;       // ring depth per worker
+    int win;          // X' window capacity in groups per token
     int n_tiles;      // 128-column tiles
-    int kh;           // consumer warps per 32-column slab
-    int stages;
-    int xpro_bytes;
-    int gmeta_bytes;
-    int recv_bytes;
-    size_t smem;
+    size_t smem;      // fixed dynamic shared-memory footprint
 };
 bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *plan);
+size_t gemv_part_bytes(int M);
 cudaError_t configure_gemv();
 cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __half *X,
                         const __half *s, const __half *scales, const int32_t *zeros, __half *Y,
-                        int M, int K, int N, int32_t *status, cudaStream_t st);
+                        int M, int K, int N, uint32_t *counters, float *part, int32_t *status,
+                        cudaStream_t st);
 
 // matmul_small.cu -- M < 64: register-fed tensor cores, TMA weight stream
 struct SmallMPlan {
@@ -79,6 +80,26 @@ cudaError_t configure_tcs();
 cudaError_t launch_tcs(const TcsPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
                        const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                        int32_t *status, cudaStream_t st);
+
+// search.cu -- scale search over alpha: scales of one grid point, transpose,
+// unquantized X W (tcgen05, float out), fixed-order loss, argmin
+size_t loss_partial_bytes();
+cudaError_t configure_search();
+cudaError_t launch_scales_alpha(const float *m, int K, int j, const int32_t *jptr, uint16_t *s, int32_t *status,
+                                cudaStream_t st);
+cudaError_t launch_transpose(const uint16_t *W, int K, int N, uint16_t *WT, cudaStream_t st);
+cudaError_t launch_dense_gemm(const CUtensorMap &tmX, const CUtensorMap &tmWT, float *Y, int R, int K, int N,
+                              int32_t *status, cudaStream_t st);
+cudaError_t launch_sq_err(const __half *Yq, const float *Yr, int64_t n, double *partial, double *loss,
+                          cudaStream_t st);
+cudaError_t launch_pick_best(const double *losses, int32_t *j_best, cudaStream_t st);
+
+// clip.cu -- weight clipping: per (group, column) the range shrink with the
+// smallest output error on calibration rows, then its codes
+cudaError_t configure_clip();
+cudaError_t launch_clip(const __half *W, const __half *s, const __half *xcal, int R, int K, int N, int n_cand,
+                        int32_t *Q, __half *scales, int32_t *zeros, int32_t *ratio, int32_t *status,
+                        cudaStream_t st);
 
 // abi.cu -- host-side argument checks of the matmul (null, shape, alignment)
 awq_status_t matmul_args_status(const uint16_t *X, const uint16_t *s, const int32_t *Q,

@@ -346,13 +346,6 @@ cudaError_t configure_small_m()
     return cudaSuccess;
 }
 
-#ifdef AWQ_TUNING
-static int tune_env(const char *name, int dflt)
-{
-    const char *v = getenv(name);
-    return v ? atoi(v) : dflt;
-}
-#endif
 
 SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
 {
@@ -372,12 +365,6 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
     // one wave: the largest power-of-two split with n_tiles * splits <= CTAs resident
     int splits = 1;
     while (splits * 2 <= max_pow2 && pl.n_tiles * splits * 2 <= (per_sm < 1 ? 1 : per_sm) * num_sms) splits *= 2;
-#ifdef AWQ_TUNING
-    splits = tune_env("AWQ_TUNE_SPLITS", splits);
-    if (splits > max_pow2) splits = max_pow2;
-    if (splits < 1) splits = 1;
-    while (splits & (splits - 1)) --splits;
-#endif
     pl.splits = splits;
     pl.smem = smem;
     return pl;

@@ -17,9 +17,10 @@
 //   warp 0      TMA ring (4 stages): X' tile [Nt tokens x 64 k] (128-byte
 //               swizzle; tokens beyond M read as zero), packed words
 //               [8 x 128]; cp.async of the group's steps and zero words.
-//   warp 1      allocates 64 TMEM columns; one lane issues
-//               tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = Nt, K = 16)
-//               x 4 per stage and commits each stage back to both rings.
+//   warp 1      allocates 256 TMEM columns (four accumulators); one lane
+//               issues tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = Nt,
+//               K = 16) x 4 per stage, k-step j into accumulator j, and commits
+//               each stage back to both rings.
 //   warps 2..9  dequantize: each writes (q - z) * step for 32 columns x 32 k
 //               as binary16 into the K-major, 128-byte-swizzled A operand
 //               (4-slot ring); then read the accumulator (tcgen05.ld) and push
@@ -37,20 +38,19 @@ namespace {
 
 constexpr int kBN = 128;               // output columns per CTA (MMA M)
 constexpr int kBK = 64;                // k per stage
-#ifndef TCS_LOAD_STAGES
-#define TCS_LOAD_STAGES 4
-#endif
-#ifndef TCS_A_STAGES
-#define TCS_A_STAGES 4
-#endif
-constexpr int kLoadStages = TCS_LOAD_STAGES;
-constexpr int kAStages = TCS_A_STAGES;  // dequantized A operand
+constexpr int kLoadStages = 4;
+constexpr int kAStages = 4;  // dequantized A operand
 constexpr int kDequantWarps = 8;
 constexpr int kThreads = 64 + 32 * kDequantWarps;
 constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 4 KB of packed words
 constexpr int kMetaBytes = 1024;              // 256 B steps + 64 B zero words, padded
 constexpr int kABytes = kBN * kBK * 2;        // 16 KB
-constexpr int kTmemCols = 64;
+// Four accumulators of up to 64 token columns: k-step j of every stage adds
+// into accumulator j, so four independent tcgen05.mma chains are in flight
+// instead of one; the epilogue adds them in the fixed order 0, 1, 2, 3.
+constexpr int kAccs = kBK / 16;
+constexpr int kAccCols = 64;
+constexpr int kTmemCols = kAccs * kAccCols;
 
 struct Params {
     const __half *scales;
@@ -180,8 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b0 = smem_u32(smem + st * p.stage_bytes);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
-                    tc_mma(tmem_base, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
-                           (i > 0 || k > 0) ? 1u : 0u);
+                    tc_mma(tmem_base + k * kAccCols, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
+                           i > 0 ? 1u : 0u);
                 tc_commit(&empty_load[st]);
                 tc_commit(&empty_a[as]);
             }
@@ -261,11 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
         const uint32_t rbase = map_to_rank(smem_u32(recv), owner);
         for (int t0 = tb; t0 < tb + p.nt / 2; t0 += 8) {
-            uint32_t v[8];
-            tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + t0, v);
+            float sum[8];
+#pragma unroll
+            for (int a = 0; a < kAccs; ++a) {
+                uint32_t v[8];
+                tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * kAccCols + t0, v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sum[j] = a == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float x = have_acc ? __uint_as_float(v[j]) : 0.0f;
+                const float x = have_acc ? sum[j] : 0.0f;
                 const int off = ((split * p.nt + t0 + j) * cpo + lc) * 4;
                 st_async_f32(rbase + off, x, rbar);
             }
@@ -307,13 +313,6 @@ TcsPlan plan_tcs(int M, int K, int N, int num_sms)
     // and leaves every CTA at least four stages.
     int splits = 1;
     while (splits * 2 <= 8 && pl.n_tiles * splits * 2 <= 2 * num_sms && KB / (splits * 2) >= 4) splits *= 2;
-#ifdef AWQ_TUNING
-    if (const char *v = getenv("AWQ_TUNE_TCS_SPLITS")) {
-        int s = atoi(v);
-        while (s > 1 && (s & (s - 1))) --s;
-        if (s >= 1 && s <= 8 && KB / s >= 1) splits = s;
-    }
-#endif
     pl.splits = splits;
     pl.stage_bytes = pl.nt * 128 + kQBytes + kMetaBytes;
     pl.smem = 1024 + static_cast<size_t>(kLoadStages) * pl.stage_bytes + static_cast<size_t>(kAStages) * kABytes +

@@ -78,22 +78,6 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
 }
 
 // ------------------------------------------------------------------ compute_scales
-// Round a positive finite double to the nearest binary16, ties to even, in a
-// single rounding (IEEE 754 binary16: quantum 2^(e-10) in the binade
-// [2^e, 2^(e+1)), never finer than the subnormal quantum 2^-24).
-__device__ uint16_t double_to_half_rn(double x)
-{
-    if (!(x < 65520.0)) return 0x7C00;  // rounds to +inf (x >= 65520)
-    if (x == 0.0) return 0;
-    const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x));
-    int e = static_cast<int>((b >> 52) & 0x7FF) - 1023;  // x normal in double here
-    int q = e - 10;
-    if (q < -24) q = -24;
-    const double inv_quantum = __longlong_as_double(static_cast<long long>(1023 - q) << 52);
-    const double n = rint(__dmul_rn(x, inv_quantum));  // exact scaling, then RNE
-    return static_cast<uint16_t>(((q + 24) << 10) + static_cast<int>(n));
-}
-
 __device__ __forceinline__ double scale_t(float mk)
 {
     return __dsqrt_rn(fmax(static_cast<double>(mk), 1e-8));
