@@ -202,8 +202,7 @@ AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s
  * awq_w4a16_gemv is the M = 1 (single-token decode) entry point:
  *   X binary16 [1, K], Y binary16 [1, N].
  * awq_w4a16_gemm takes any 1 <= M <= AWQ_MAX_M and picks its tile path
- * internally: the decode GEMV for M <= 2 (persistent, one CTA per SM, split
- * tiles finished by the last-arriving worker), register-fed tensor cores for
+ * internally: the decode GEMV for M <= 2, register-fed tensor cores for
  * 3 <= M < 40, tcgen05/TMEM for M >= 40 (small batch from 40, prefill from 64).
  *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack;
  *   zeros = NULL for weights from awq_quantize_pack_symmetric (zero point 8).
@@ -213,9 +212,9 @@ AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s
  *   the call with the original X and s.
  * Workspace: caller-owned device memory of at least *_workspace_size() bytes,
  * never NULL.  It must be zero-filled (e.g. cudaMemsetAsync) before its first
- * use: its first 32 KB hold arrival counters that a call expects at zero and
+ * use: its first 32 KB are a counter block that a call expects at zero and
  * leaves at zero when it completes without a device error.  The rest holds
- * X / s and partial sums and is overwritten.  Calls on one stream may share a
+ * X / s and is overwritten.  Calls on one stream may share a
  * workspace; calls that can run at the same time need separate ones.  After a
  * device error (AWQ_ERR_DEVICE_TIMEOUT) zero the workspace again.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
@@ -315,8 +314,8 @@ AWQ_API awq_status_t awq_scale_search(const uint16_t *xcal, int64_t R, int64_t K
  *
  * Arguments, layouts, tolerance and errors are those of awq_w4a16_gemm, minus
  * the workspace.  Limit: awq_w4a16_gemm_workspace_size(M, K, N) must not exceed
- * AWQ_NOALLOC_SCRATCH_BYTES (32 KB of counters + 2 * M * K bytes of X / s, plus
- * 768 KB per token for M <= 2; for example M * K <= 2 Mi elements at M >= 3);
+ * AWQ_NOALLOC_SCRATCH_BYTES (32 KB of counters + 2 * M * K bytes of X / s, i.e.
+ * M * K <= 2 Mi - 16 Ki elements);
  * larger problems return AWQ_ERR_WORKSPACE before anything runs.
  * Set-up: the first call on each device (with that device current) looks up
  * the scratch array's device address; make that first call before any stream

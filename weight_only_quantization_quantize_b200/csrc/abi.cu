@@ -155,19 +155,18 @@ bool matmul_shape_ok(int64_t M, int64_t K, int64_t N)
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace layout of every matmul call:
-//   [0, 32 KB)              arrival counters of the split tiles (one uint32 per
-//                           128-column tile, up to AWQ_MAX_N / 128); zero
-//                           between calls: each call resets what it used
+//   [0, 32 KB)              a counter block (one uint32 per 128-column tile, up
+//                           to AWQ_MAX_N / 128) reserved for kernels that
+//                           count arrivals on shared tiles; zero between calls
 //   [32 KB, +2MK)           X / s (binary16, pair-permuted) for the small-batch
 //                           and tcgen05 paths
-//   then, for M <= 2        the decode GEMV's float partials of split tiles
 constexpr size_t kCounterBytes = static_cast<size_t>(AWQ_MAX_N / 128) * sizeof(uint32_t);
 
 size_t xp_bytes(int64_t M, int64_t K) { return round_up(static_cast<size_t>(2 * M * K), 256); }
 
 size_t workspace_bytes(int64_t M, int64_t K)
 {
-    return kCounterBytes + xp_bytes(M, K) + (M <= 2 ? awq::gemv_part_bytes(static_cast<int>(M)) : 0);
+    return kCounterBytes + xp_bytes(M, K);
 }
 
 awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
@@ -194,21 +193,18 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
     const __half *hsc = reinterpret_cast<const __half *>(scales);
     __half *hY = reinterpret_cast<__half *>(Y);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    uint32_t *counters = reinterpret_cast<uint32_t *>(wsb);
     __half *Xp = reinterpret_cast<__half *>(wsb + kCounterBytes);
-    float *part = reinterpret_cast<float *>(wsb + kCounterBytes + xp_bytes(M, K));
 
     CUtensorMap tmQ, tmX;
     awq::GemvPlan gplan;
-    // The decode GEMV (X / s and its group sums in shared memory) for one or
-    // two tokens; from three tokens on, the small-batch kernels with the X / s
-    // pre-pass (measured faster on the 7B and 13B layer shapes).
+    // The decode GEMV (X / s and its group sums in shared memory) wins for one
+    // or two tokens; from three tokens on, the small-batch kernel with the
+    // X / s pre-pass is faster (measured on the 7B and 13B layer shapes).
     if (M <= 2 && awq::plan_gemv(m, k, n, sms, &gplan)) {
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;
-        return from_cuda(awq::launch_gemv(gplan, tmQ, hX, hs, hsc, zeros, hY, m, k, n, counters, part,
-                                          dev_status, st));
+        return from_cuda(awq::launch_gemv(gplan, tmQ, hX, hs, hsc, zeros, hY, m, k, n, dev_status, st));
     }
     // From about 40 tokens the small-batch layer needs more MMA rate than
     // mma.sync gives: tcgen05 with the weights as the 128-row operand

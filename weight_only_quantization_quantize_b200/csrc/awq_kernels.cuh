@@ -19,23 +19,22 @@ cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K,
 cudaError_t launch_fold_inverse_scale(const __half *a, int64_t rows, int K, const __half *s,
                                       __half *out, int32_t *status, int num_sms, cudaStream_t st);
 
-// gemv.cu -- M <= 2: decode GEMV, persistent stream-K over (tile, group)
-// units, zero point and step applied once per group
-constexpr int kGemvMaxCtas = 256;  // upper bound of the persistent grid
+// gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group
 struct GemvPlan {
-    int ctas;         // persistent CTAs (at most one per SM)
-    int stages;       // ring depth per worker
-    int win;          // X' window capacity in groups per token
+    int splits;       // CTAs per cluster along K
     int n_tiles;      // 128-column tiles
-    size_t smem;      // fixed dynamic shared-memory footprint
+    int kh;           // consumer warps per 32-column slab
+    int stages;
+    int xpro_bytes;
+    int gmeta_bytes;
+    int recv_bytes;
+    size_t smem;
 };
 bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *plan);
-size_t gemv_part_bytes(int M);
 cudaError_t configure_gemv();
 cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __half *X,
                         const __half *s, const __half *scales, const int32_t *zeros, __half *Y,
-                        int M, int K, int N, uint32_t *counters, float *part, int32_t *status,
-                        cudaStream_t st);
+                        int M, int K, int N, int32_t *status, cudaStream_t st);
 
 // matmul_small.cu -- M < 64: register-fed tensor cores, TMA weight stream
 struct SmallMPlan {
