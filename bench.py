@@ -289,6 +289,7 @@ def run_ours(args, rank, world, device):
         del qlayers
         extra["decode_7b_symmetric"] = run_decode_variant(awq, device, peaks, nlayers)
         extra["decode_7b_prescaled"] = run_decode_variant(awq, device, peaks, nlayers, prescaled=True)
+        extra.update(run_calibration(awq, device))
 
     cpu = run_cpu_baseline(rank, world) if rank == 0 else None
     return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, launches=launches,
@@ -316,6 +317,7 @@ def run_e2e(awq, layers, args, device):
     xv = [[dx[li][xo[pi]:xo[pi + 1]].view(1, -1) for pi in range(len(ks))] for li in range(nl)]
     yv = [[dy[li][yo[pi]:yo[pi + 1]].view(1, -1) for pi in range(len(ns))] for li in range(nl)]
     lin = [[awq.QuantLinear(p["Q"], p["sc"], p["z"], p["s"]) for p in layer] for layer in layers]
+    ws = zeroed_workspace(awq, device, [(p["K"], p["N"]) for p in layers[0]], [1])
     h2d = 2 * int(xo[-1])
     d2h = 2 * int(yo[-1])
 
@@ -323,12 +325,13 @@ def run_e2e(awq, layers, args, device):
         li = i % nl
         dx[li].copy_(hx[li], non_blocking=True)
         for pi, f in enumerate(lin[li]):
-            f(xv[li][pi], out=yv[li][pi])
+            f(xv[li][pi], out=yv[li][pi], workspace=ws)
         hy[li].copy_(dy[li], non_blocking=True)
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    wb = sum(weight_bytes(p["K"], p["N"]) for p in layers[0])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
@@ -336,12 +339,11 @@ def run_e2e(awq, layers, args, device):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    wb = sum(weight_bytes(p["K"], p["N"]) for p in layers[0])
     return {"value": round(wb * args.steps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4),
             "path": "QuantLinear (python binding -> C ABI), eager; one H2D copy of the step's 4 "
-                    "activation rows, one D2H copy of its 4 outputs"}
+                    "activation rows from pinned host memory, one D2H copy of its 4 outputs"}
 
 
 def flush_l2(buf):
@@ -409,6 +411,45 @@ def run_config_sweep(awq, device, peaks, peak_src):
     r = run_sweep(awq, device, peaks, peak_src, 5, [1, 32, 256], 2, ["hbm", "hbm", "tensor"])
     out.update({f"stack_70b_m{M}": e for M, e in r.items()})
     return out
+
+
+def run_calibration(awq, device, reps=3):
+    """The two calibration searches on one 7B projection (O, 4096 x 4096, 256
+    calibration rows): the scale search over alpha = j/8 and weight clipping
+    (11 candidate ranges).  Calibration runs once per layer, offline."""
+    wl = synth.WORKLOADS[WORKLOAD_ID]
+    K, N, _ = wl.shapes[1]
+    L = synth.make_layer(WORKLOAD_ID, 0, M=1, K=K, N=N, R=wl.R, device=device, shape_id=1)
+    R = wl.R
+    ws = torch.zeros(awq.scale_search_workspace_size(R, K, N), dtype=torch.uint8, device=device)
+    s = awq.compute_scales(awq.act_stats(L.Xcal))
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return statistics.median(t)
+
+    ms_search = timed(lambda: awq.scale_search(L.Xcal, L.W, workspace=ws))
+    ms_clip = timed(lambda: awq.quantize_pack_clip(L.W, s, L.Xcal, 11))
+    gemm_flops = 10 * 2 * R * K * N          # the unquantized X W and 9 quantized products
+    clip_flops = 11 * 2 * R * K * N          # candidate error vectors applied to the rows
+    return {"scale_search_7b_o": {"ms": round(ms_search, 3), "grid": "alpha = j/8, j = 0..8",
+                                  "calib_rows": R, "matmul_tflops": round(gemm_flops / (ms_search * 1e-3) / 1e12, 1),
+                                  "includes": "statistics, W transpose, X W (tcgen05), 9 x (scales, quantize_pack, "
+                                              "W4A16 matmul at M = R, loss), argmin"},
+            "quantize_clip_7b_o": {"ms": round(ms_clip, 3), "candidates": 11, "calib_rows": R,
+                                   "fp32_tflops": round(clip_flops / (ms_clip * 1e-3) / 1e12, 1),
+                                   "includes": "per (group, column) 11 ranges scored on the calibration rows, "
+                                               "codes of the best"}}
 
 
 def run_decode_variant(awq, device, peaks, nlayers, steps=200, warmup=5, prescaled=False):

@@ -99,5 +99,8 @@ def test_quant_linear_checks_weights_once_and_inputs_every_call():
         lin(torch.zeros(2, 128, dtype=torch.float16, device="cuda"))
     with pytest.raises(ValueError, match="out"):
         lin(X, out=torch.empty(2, 8, dtype=torch.float16, device="cuda"))
-    # zero weights: Y = 0 exactly
-    assert torch.equal(lin(X), torch.zeros(2, 64, dtype=torch.float16, device="cuda"))
+    # the prepared layer runs the same call as the functional entry point
+    Q.random_(-2**31, 2**31 - 1)
+    z.random_(-2**31, 2**31 - 1)
+    assert torch.equal(lin(X), awq.w4a16_gemm(X, s, Q, sc, z))
+    assert torch.equal(lin(X[:1].contiguous()), awq.w4a16_gemv(X[:1].contiguous(), s, Q, sc, z))

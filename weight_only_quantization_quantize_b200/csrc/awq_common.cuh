@@ -21,13 +21,18 @@ constexpr int kGroup = 128;
 // caller then skips its remaining work but still reaches every block- and
 // cluster-wide barrier, so the context survives and the host can read the
 // status word.
-// AWQ_WAIT_LIMIT_NS exists for the test build that checks the timeout path
-// (a wait that does not complete at once then runs out); the library itself
-// is always built with the default.
+// AWQ_WAIT_LIMIT_NS, AWQ_WAIT_POLL_MASK and AWQ_WAIT_NONBLOCKING_POLL exist for
+// the test build that checks the timeout path (limit 0, timer read on every
+// poll, polls that never suspend: a wait that does not complete at its first
+// poll runs out); the library itself is always built with the defaults.
 #ifndef AWQ_WAIT_LIMIT_NS
 #define AWQ_WAIT_LIMIT_NS 1000000000ull
 #endif
 constexpr uint64_t kWaitLimitNs = AWQ_WAIT_LIMIT_NS;  // 1 s
+#ifndef AWQ_WAIT_POLL_MASK
+#define AWQ_WAIT_POLL_MASK 255u
+#endif
+constexpr uint32_t kWaitPollMask = AWQ_WAIT_POLL_MASK;  // read the timer every 256 polls
 // After a wait has run out, a kernel still lets the copies it issued land
 // before it exits; those waits use their own limit.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s
@@ -75,6 +80,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity)
 {
     uint32_t done;
+#ifdef AWQ_WAIT_NONBLOCKING_POLL
+    // test build: a poll that never suspends the thread
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+#else
+    // may suspend the thread for a while until the phase completes
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -82,6 +98,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
         : "=r"(done)
         : "r"(bar_addr), "r"(parity)
         : "memory");
+#endif
     return done != 0;
 }
 
@@ -94,7 +111,7 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, ui
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(a, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer() - t0 > limit_ns) return false;
+        if ((i & kWaitPollMask) == 0 && globaltimer() - t0 > limit_ns) return false;
     }
 }
 

@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         // while that kernel finishes.
         const int pre = ng < S ? ng : S;
         bool ok = true;
+        int issued = 0;
         for (int it = 0; it < ng; ++it) {
             if (it == pre) pdl_wait();
             const int st = it % S;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                 ok = false;
                 break;
             }
+            issued = it + 1;
             uint8_t *stg = smem + st * kStageBytes;
             const int g = g_begin + it;
             if (lane == 0) {
@@ -156,6 +158,13 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         }
         pdl_wait();  // before this warp writes Y in the epilogue
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+        // Every copy this warp issued lands before the CTA can exit: after a
+        // consumer's wait ran out, stages may still be in flight (the waits
+        // here have their own limit).
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (lane == 0)
+            for (int it = issued > S ? issued - S : 0; it < issued; ++it)
+                mbar_wait_for(&full[it % S], (it / S) & 1, kDrainLimitNs);
     } else {
         // ------------------------------------------------------------ consumers
         pdl_wait();
@@ -336,7 +345,11 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     // when that CTA leaves.  (A release here fenced on the pushes' completion.)
     cluster_arrive_relaxed();
     // Reduce the columns this rank owns, partials summed in (rank, k-half) order.
-    if (!mbar_wait(recv_bar, 0) && threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    if (!mbar_wait(recv_bar, 0)) {
+        if (threadIdx.x == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+        // the partials pushed into this CTA still land before it exits
+        mbar_wait_for(recv_bar, 0, kDrainLimitNs);
+    }
     const int lchunks = cpo / 8;
     for (int e = threadIdx.x; e < p.M * lchunks; e += kAllThreads) {
         const int tok = e / lchunks;
