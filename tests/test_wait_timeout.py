@@ -67,3 +67,34 @@ def test_gemv_wait_runs_out_and_the_context_survives(waitlib):
     y = Y2.cpu().numpy().astype(np.float64)
     assert np.abs(y - Yr).max() <= 1e-2 * np.abs(Yr).max()
     assert np.linalg.norm(y - Yr) <= 5e-3 * np.linalg.norm(Yr)
+
+
+def test_prefill_wait_runs_out_and_the_context_survives(waitlib):
+    # the tcgen05 path with the weights in tensor memory: 16 stages of 64 k per
+    # tile against a 5-deep load ring, so the producer has to wait for a slot
+    M, K, N = 256, 1024, 512
+    waitlib.awq_w4a16_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P, SZ, P, P]
+    waitlib.awq_w4a16_gemm.restype = ctypes.c_int
+    L = synth.make_layer(19, 0, M=M, K=K, N=N, R=64)
+    s = awq.compute_scales(awq.act_stats(L.Xcal.cuda()))
+    Q, sc, z = awq.quantize_pack(L.W.cuda(), s)
+    X = L.X.cuda()
+    ws = torch.zeros(awq.gemm_workspace_size(M, K, N), dtype=torch.uint8, device="cuda")
+    Y = torch.zeros(M, N, dtype=torch.float16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = waitlib.awq_w4a16_gemm(X.data_ptr(), s.data_ptr(), Q.data_ptr(), sc.data_ptr(), z.data_ptr(), M, K, N,
+                                Y.data_ptr(), ws.data_ptr(), ws.numel(), st.data_ptr(), stream)
+    assert rc == awq.OK
+    torch.cuda.synchronize()              # the kernel finished: no hang, no fault
+    assert int(st.item()) == awq.ERR_TIMEOUT
+    st2 = awq.new_status("cuda")
+    Y2 = awq.w4a16_gemm(X, s, Q, sc, z, status=st2)
+    awq.raise_on_status(st2, "prefill matmul after a timed-out call")
+    sr = s.cpu().numpy()
+    Qr, scr, zr = oracle.quantize_pack(L.W.numpy(), sr)
+    Yr = oracle.matmul(L.X.numpy(), sr, Qr, scr, zr, precision=64, nthreads=16)
+    y = Y2.cpu().numpy().astype(np.float64)
+    assert np.abs(y - Yr).max() <= 1e-2 * np.abs(Yr).max()
+    assert np.linalg.norm(y - Yr) <= 5e-3 * np.linalg.norm(Yr)

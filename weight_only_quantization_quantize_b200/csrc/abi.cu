@@ -4,7 +4,7 @@
 // one-time per-device architecture check, TMA descriptor encoding, workspace
 // accounting and the choice of tile path.  Every step of the computation runs
 // in the kernels of quantize.cu, fold.cu, gemv.cu, matmul_small.cu,
-// matmul_tcs.cu and matmul_tc.cu.
+// matmul_tcs.cu and matmul_tct.cu.
 #include <mutex>
 
 #include "awq_kernels.cuh"
@@ -68,7 +68,7 @@ awq_status_t device_ready(int *sms)
                 }
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
-            if (awq::configure_tc() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
+            if (awq::configure_tct() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
                 awq::configure_gemv() != cudaSuccess || awq::configure_quantize() != cudaSuccess ||
                 awq::configure_tcs() != cudaSuccess || awq::configure_search() != cudaSuccess ||
                 awq::configure_clip() != cudaSuccess) {
@@ -233,15 +233,15 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         return from_cuda(awq::launch_small_m(plan, tmQ, tmX, hX, hs, hsc, zeros, hY, m, k, n,
                                              dev_status, st));
     }
-    const awq::TcPlan plan = awq::plan_tc(m, k, n, sms);
-    if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64, 128,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 256, 8,
+    const awq::TctPlan plan = awq::plan_tct(m, k, n, sms);
+    if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
+                   static_cast<uint32_t>(plan.bt), CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 8,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return AWQ_ERR_CUDA;
     e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
     if (e != AWQ_OK) return e;
-    return from_cuda(awq::launch_tc(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
+    return from_cuda(awq::launch_tct(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
 }
 
 }  // namespace

@@ -55,16 +55,18 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
                            const int32_t *zeros, __half *Y, int M, int K, int N,
                            int32_t *status, cudaStream_t st);
 
-// matmul_tc.cu -- M >= 64: tcgen05 / TMEM
-struct TcPlan {
+// matmul_tct.cu -- M >= 64: tcgen05 with the dequantized weights in TMEM
+// (transposed tile: 128 output columns x bt tokens)
+struct TctPlan {
+    int bt;        // tokens per tile: 128 or 256
     int m_tiles, n_tiles;
     size_t smem;
 };
-TcPlan plan_tc(int M, int K, int N, int num_sms);
-cudaError_t configure_tc();
-cudaError_t launch_tc(const TcPlan &plan, const CUtensorMap &tmA, const CUtensorMap &tmQ,
-                      const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
-                      int32_t *status, cudaStream_t st);
+TctPlan plan_tct(int M, int K, int N, int num_sms);
+cudaError_t configure_tct();
+cudaError_t launch_tct(const TctPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
+                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                       int32_t *status, cudaStream_t st);
 
 // matmul_tcs.cu -- 40 <= M < 64: tcgen05 with the weights as the 128-row operand
 struct TcsPlan {
