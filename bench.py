@@ -598,7 +598,7 @@ def run_profile(workload, M, reps):
         L = synth.make_layer(workload, 0, M=M, K=K, N=N, R=wl.R, device="cuda", shape_id=si)
         s = awq.compute_scales(awq.act_stats(L.Xcal))
         Q, sc, z = awq.quantize_pack(L.W, s)
-        ws = torch.empty(max(awq.gemm_workspace_size(M, K, N), 16), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(max(awq.gemm_workspace_size(M, K, N), 16), dtype=torch.uint8, device="cuda")
         projs.append((L.X, s, Q, sc, z, ws))
         del L
     torch.cuda.synchronize()

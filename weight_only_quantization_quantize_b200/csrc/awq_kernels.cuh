@@ -19,11 +19,10 @@ cudaError_t launch_quantize_pack(const CUtensorMap &tmW, const __half *s, int K,
 cudaError_t launch_fold_inverse_scale(const __half *a, int64_t rows, int K, const __half *s,
                                       __half *out, int32_t *status, int num_sms, cudaStream_t st);
 
-// gemv.cu -- M <= 8: decode GEMV, zero point and step applied once per group
+// gemv.cu -- M <= 2: decode GEMV, zero point and step applied once per group
 struct GemvPlan {
     int splits;       // CTAs per cluster along K
     int n_tiles;      // 128-column tiles
-    int kh;           // consumer warps per 32-column slab
     int stages;
     int xpro_bytes;
     int gmeta_bytes;

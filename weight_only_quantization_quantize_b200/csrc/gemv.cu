@@ -1,5 +1,5 @@
-// gemv.cu -- Y = (X / s) . dequant(Q) for M <= 8 tokens: the single-token
-// decode GEMV (and the smallest batches), the HBM-bound regime.
+// gemv.cu -- Y = (X / s) . dequant(Q) for M <= 2 tokens: the single-token
+// decode GEMV (and two-token steps), the HBM-bound regime.
 //
 // Sources: lansai AWQ explainer (ai.lansai.wang/107648), "AWQ 的四步链路"
 // (Y = (X/s)(sW)); "Awq Quantization" (skillselion.com), "WQLinear Kernel
@@ -8,22 +8,28 @@
 //
 // Every packed weight is read once from HBM.  To keep the per-weight work at a
 // handful of integer ops, the zero point and the step leave the inner loop:
-// with S0 / S1 the sums of X' over the group's even / odd k (k mod 8), and
-// R0 = sum_{k even} x'_k (1024 + q_k),  R1 = sum_{k odd} x'_k (1024 + 16 q_k)
-// (what the tensor cores produce when fed the raw OR-ed nibbles),
-//   sum_k x'_k (q_k - z) = R0 + R1 / 16 - (1024 S0 + 64 S1) - z (S0 + S1),
+// the tensor cores are fed the raw OR-ed nibbles (1024 + q_k for even k mod 8,
+// 1024 + 16 q_k for odd k) against x'_k and x'_k / 16, so that with S0 / S1
+// the sums of those x' over the group's even / odd k,
+//   R = sum_{k even} x'_k (1024 + q_k) + sum_{k odd} (x'_k / 16)(1024 + 16 q_k)
+//   sum_k x'_k (q_k - z) = R - (1024 S0 + 64 S1) - z (S0 + S1),
 // and the group's step multiplies that once.  S0, S1 are computed per CTA in
 // the prologue together with X' = fp16(X / s), from the same rounded values.
+//
+// The MMA (m16n8k16, swap-AB: columns are MMA rows) has 8 token columns; with
+// one or two tokens, the spare columns carry further groups: column c of the
+// accumulator is (group c / M of a batch of 8 / M groups, token c % M).  A
+// lane's B operand is X' where its column's group is the stage's group and
+// zero elsewhere, so one accumulator fragment collects a whole batch and the
+// step / zero point arithmetic runs once per batch instead of once per group.
 //
 // Structure (one CTA = 128 output columns x a k range; clusters split K):
 //   producer warp   TMA ring of 128-row groups (four 16 x 32-word boxes,
 //                   128-byte swizzle) + cp.async of the group's steps and zero
 //                   words; ring depth 8, 6 or 4 (see plan_gemv).
-//   4*KH consumers  32 columns per warp (KH warps split a group's rows); a
-//                   lane turns one 16-byte load (4 columns x 8 k) into four
-//                   even-form and four odd-form f16x2 operands with LOP3 only
-//                   and feeds mma.sync m16n8k16 in swap-AB form (columns are
-//                   MMA rows, tokens MMA columns).
+//   4 consumers     32 columns per warp; a lane turns one 16-byte load
+//                   (4 columns x 8 k) into four even-form and four odd-form
+//                   f16x2 operands with LOP3 only and feeds mma.sync.
 //   epilogue        each CTA pushes its partial columns into the shared memory
 //                   of the cluster CTA that owns them (st.async, completion as
 //                   transaction bytes on the owner's mbarrier); owners sum the
@@ -38,6 +44,7 @@ constexpr int kBN = 128;
 constexpr int kQStage = 4 * 2048;
 constexpr int kStageBytes = 9216;  // 8 KB words + 256 B steps + 64 B zero words, padded
 constexpr int kSmemOptIn = 232448;
+constexpr int kConsumers = 4;  // one warp per 32-column slab of the 128-column tile
 
 struct GemvParams {
     const __half *X;
@@ -64,14 +71,18 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <int S, int KH>
-__global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
+template <int S, int MT>
+__global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmQ, const GemvParams p)
 {
-    constexpr int kConsumers = 4 * KH;
     constexpr int kCThreads = 32 * kConsumers;
     constexpr int kAllThreads = kCThreads + 32;
-    constexpr int kSteps = 4 / KH;
+    // The MMA's 8 token columns carry (group, token) slots: slot = MT * (group
+    // within a batch of kGPB groups) + token, so one accumulator fragment holds
+    // kGPB groups' sums and the step / zero point are applied once per batch.
+    constexpr int kGPB = 8 / MT;
+    constexpr int kLG = 2 / MT;  // groups among a lane's two fragment columns
+    static_assert(MT == 1 || MT == 2, "the decode GEMV takes one or two tokens");
 
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *smem = align1024(smem_dyn);
@@ -102,7 +113,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         mbar_init(recv_bar, 1);
         fence_barrier_init();
         // expect every rank's partials for the columns this CTA owns
-        mbar_arrive_expect_tx(recv_bar, KH * p.M * cpo * p.splits * 4);
+        mbar_arrive_expect_tx(recv_bar, MT * cpo * p.splits * 4);
     }
     __syncthreads();
     // Barriers initialized; waited on before the first push.  The init fence
@@ -170,9 +181,11 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
         pdl_wait();
         // Prologue: X' = fp16(X / s) for this CTA's k range, stored per 8-channel
         // chunk in the order (0,4),(2,6),(1,5),(3,7) (even-form pairs, then
-        // odd-form pairs), plus the per-(token, group, half) sums of X'.
+        // odd-form pairs), the odd-form values divided by 16 (exact unless the
+        // quotient is subnormal, and the sums below use the same rounded
+        // values), plus the per-(token, group) sums of X'.
         {
-            constexpr int kLanesPerHalf = 16 / KH;  // chunks per group half
+            constexpr int kLanesPerGroup = 16;  // 8-channel chunks per group
             const int sub = lane >> 4;              // two (token, group) pairs per warp pass
             const int c16 = lane & 15;
             const int pairs = p.M * ng;
@@ -208,10 +221,12 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                         const __half *sh = reinterpret_cast<const __half *>(&sv[b]);
                         __half q[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
+                        for (int j = 0; j < 8; ++j) {
                             q[j] = __float2half_rn(__fdiv_rn(__half2float(xh[j]), __half2float(sh[j])));
+                            if (j & 1) q[j] = __float2half_rn(__half2float(q[j]) * 0.0625f);
+                        }
                         e = (__half2float(q[0]) + __half2float(q[2])) + (__half2float(q[4]) + __half2float(q[6]));
-                        o = (__half2float(q[1]) + __half2float(q[3])) + (__half2float(q[5]) + __half2float(q[7]));
+                        o = 16.0f * ((__half2float(q[1]) + __half2float(q[3])) + (__half2float(q[5]) + __half2float(q[7])));
                         uint4 r;
                         r.x = __half_as_ushort(q[0]) | (static_cast<uint32_t>(__half_as_ushort(q[4])) << 16);
                         r.y = __half_as_ushort(q[2]) | (static_cast<uint32_t>(__half_as_ushort(q[6])) << 16);
@@ -219,15 +234,14 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                         r.w = __half_as_ushort(q[3]) | (static_cast<uint32_t>(__half_as_ushort(q[7])) << 16);
                         *reinterpret_cast<uint4 *>(xpro + (static_cast<size_t>(tok[b]) * chunks + (ch ^ (tok[b] & 7))) * 16) = r;
                     }
-                    // butterfly over the lanes of one group half (fixed order)
+                    // butterfly over the lanes of one group (fixed order)
 #pragma unroll
-                    for (int off = kLanesPerHalf / 2; off > 0; off >>= 1) {
+                    for (int off = kLanesPerGroup / 2; off > 0; off >>= 1) {
                         e += __shfl_xor_sync(0xffffffffu, e, off);
                         o += __shfl_xor_sync(0xffffffffu, o, off);
                     }
-                    if (valid[b] && (c16 % kLanesPerHalf) == 0)
-                        gmeta[(tok[b] * ng + gl[b]) * KH + c16 / kLanesPerHalf] =
-                            make_float2(fmaf(1024.0f, e, 64.0f * o), e + o);
+                    if (valid[b] && c16 == 0)
+                        gmeta[tok[b] * ng + gl[b]] = make_float2(fmaf(1024.0f, e, 64.0f * o), e + o);
                 }
             }
             named_bar_sync(1, kCThreads);
@@ -235,42 +249,54 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 
         const int gq = lane >> 2;
         const int t = lane & 3;
-        const int slab = warp & 3;
-        const int khalf = warp >> 2;
-        const int colw = 32 * slab + 4 * gq;
-        const int tok0 = 2 * t;
-        // This lane's X' row (tokens beyond M never load it).  A chunk index
-        // it * 16 + r XOR-swizzled by gq < 8 equals it * 16 + (r ^ gq).
-        const uint8_t *xrow = xpro + static_cast<size_t>(gq) * chunks * 16;
+        const int colw = 32 * warp + 4 * gq;  // this lane's 4 columns (A rows gq, gq + 8 of 2 tiles)
+        // This lane's B column (MMA token column gq) is slot gq: group gq / MT
+        // of each batch, token gq % MT.  Its accumulator columns 2t, 2t + 1
+        // are slots of group(s) (2t) / MT, (2t + 1) / MT.
+        const int b_group = gq / MT;
+        const int b_tok = gq % MT;
+        // This lane's X' row.  A chunk index it * 16 + r XOR-swizzled by the
+        // token (< 8) equals it * 16 + (r ^ token).
+        const uint8_t *xrow = xpro + static_cast<size_t>(b_tok) * chunks * 16;
         const uint32_t mlo = p.mask_lo, mhi = p.mask_hi, magic = p.magic;
+        float R[2][4];  // [tile][fragment element], one batch of groups
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) R[a][i] = 0.0f;
+        // steps (4 binary16) and zero word of the group(s) this lane finishes
+        // (two named sets rather than an array: a run-time index would put
+        // the array in local memory)
+        uint2 cap_sc0 = make_uint2(0u, 0u), cap_sc1 = cap_sc0;
+        uint32_t cap_z0 = 0u, cap_z1 = 0u;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
             const int st = it % S;
-            if (!mbar_wait(&full[st], (it / S) & 1)) {
+            const int j = it % kGPB;  // group within the batch
+            // the outcome is voted so that the warp leaves the loop as one
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (it / S) & 1))) {
                 ok = false;
                 break;
             }
             const uint8_t *stg = smem + st * kStageBytes;
             const uint8_t *meta = stg + kQStage;
-            const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
-            const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
-
-            float R[2][2][4];  // [tile][form][c]
+            if (t == j / kLG) {
+                const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
+                const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
+                const bool second = kLG == 2 && (j & 1);
+                cap_sc0 = second ? cap_sc0 : sc;
+                cap_z0 = second ? cap_z0 : zw;
+                cap_sc1 = second ? sc : cap_sc1;
+                cap_z1 = second ? zw : cap_z1;
+            }
+            const bool mine = b_group == j;
+            const uint8_t *qslab = stg + warp * 2048;
 #pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int f = 0; f < 2; ++f)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) R[a][f][i] = 0.0f;
-
-            const uint8_t *qslab = stg + slab * 2048;
-#pragma unroll
-            for (int ss = 0; ss < kSteps; ++ss) {
-                const int sidx = khalf * kSteps + ss;
-                const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);
+            for (int ss = 0; ss < 4; ++ss) {
+                const int r = 8 * (ss >> 1) + 2 * t + (ss & 1);
                 const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
                 uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-                if (gq < p.M) bx = *reinterpret_cast<const uint4 *>(xrow + it * 256 + ((r ^ gq) << 4));
+                if (mine) bx = *reinterpret_cast<const uint4 *>(xrow + it * 256 + ((r ^ b_tok) << 4));
                 const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
                 uint32_t ev0[4], ev2[4], od1[4], od3[4];
 #pragma unroll
@@ -286,33 +312,62 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
                     const int c0 = 2 * tile, c1 = 2 * tile + 1;
                     const uint32_t ae[4] = {ev0[c0], ev0[c1], ev2[c0], ev2[c1]};
                     const uint32_t ao[4] = {od1[c0], od1[c1], od3[c0], od3[c1]};
-                    mma_16816(R[tile][0], ae, bx.x, bx.y);
-                    mma_16816(R[tile][1], ao, bx.z, bx.w);
+                    mma_16816(R[tile], ae, bx.x, bx.y);
+                    mma_16816(R[tile], ao, bx.z, bx.w);  // X' / 16 on the odd form
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
 
-            // group epilogue: y += step * (R0 + R1/16 - (1024 S0 + 64 S1) - z (S0 + S1))
-            const float2 gm0 = tok0 < p.M ? gmeta[(tok0 * ng + it) * KH + khalf] : make_float2(0.f, 0.f);
-            const float2 gm1 = tok0 + 1 < p.M ? gmeta[((tok0 + 1) * ng + it) * KH + khalf] : make_float2(0.f, 0.f);
-            const int zsh = (colw & 7) * 4;
-            const __half2 s01 = *reinterpret_cast<const __half2 *>(&sc.x);
-            const __half2 s23 = *reinterpret_cast<const __half2 *>(&sc.y);
-            const float stp[4] = {__low2float(s01), __high2float(s01), __low2float(s23), __high2float(s23)};
+            if (j == kGPB - 1 || it == ng - 1) {
+                // batch epilogue: fragment column 2t + u is slot 2t + u = group
+                // g = (2t + u) / MT of the batch, token (2t + u) % MT;
+                // y += step * (R - (1024 S0 + 64 S1) - z (S0 + S1))
+                const int base = it - j;
 #pragma unroll
-            for (int tile = 0; tile < 2; ++tile)
+                for (int u = 0; u < 2; ++u) {
+                    const int slot = 2 * t + u;
+                    const int gb = slot / MT;
+                    const int tk = slot % MT;
+                    const bool second = kLG == 2 && u == 1;
+                    const bool valid = gb <= j;
+                    const float2 gm = valid ? gmeta[tk * ng + base + gb] : make_float2(0.f, 0.f);
+                    const uint2 sc = second ? cap_sc1 : cap_sc0;
+                    const uint32_t zw = second ? cap_z1 : cap_z0;
+                    const float stp[4] = {__half2float(__ushort_as_half(static_cast<unsigned short>(sc.x & 0xFFFFu))),
+                                          __half2float(__ushort_as_half(static_cast<unsigned short>(sc.x >> 16))),
+                                          __half2float(__ushort_as_half(static_cast<unsigned short>(sc.y & 0xFFFFu))),
+                                          __half2float(__ushort_as_half(static_cast<unsigned short>(sc.y >> 16)))};
+                    const int zsh = (colw & 7) * 4;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int c = 2 * tile + (i >> 1);
-                    // the 4-bit zero as a float: 2^23 + z exactly, minus 2^23
-                    const float z = __int_as_float(((zw >> (zsh + 4 * c)) & 15u) | 0x4B000000u) - 8388608.0f;
-                    const float2 gm = (i & 1) ? gm1 : gm0;
-                    float pgrp = fmaf(R[tile][1][i], 0.0625f, R[tile][0][i]) - gm.x;
-                    pgrp = fmaf(-z, gm.y, pgrp);
-                    acc[tile][i] = fmaf(stp[c], pgrp, acc[tile][i]);
+                    for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+                        for (int row = 0; row < 2; ++row) {
+                            const int c = 2 * tile + row;
+                            // the 4-bit zero as a float: 2^23 + z exactly, minus 2^23
+                            const float z =
+                                __int_as_float(((zw >> (zsh + 4 * c)) & 15u) | 0x4B000000u) - 8388608.0f;
+                            float pgrp = R[tile][2 * row + u] - gm.x;
+                            pgrp = fmaf(-z, gm.y, pgrp);
+                            if (valid) acc[tile][2 * row + tk] = fmaf(stp[c], pgrp, acc[tile][2 * row + tk]);
+                        }
                 }
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) R[a][i] = 0.0f;
+            }
         }
+        // Sum the lanes' group partials (fixed butterfly order): lane t = 0 of
+        // each quad then holds columns colw.. for tokens 0 .. MT - 1 in the
+        // fragment layout [tile][2 row + token] that the push below expects.
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[a][i] += __shfl_xor_sync(0xffffffffu, acc[a][i], 1);
+                acc[a][i] += __shfl_xor_sync(0xffffffffu, acc[a][i], 2);
+            }
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     }
 
@@ -322,8 +377,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     cluster_wait_acquire();  // every CTA of the cluster has initialized its barriers
     if (warp < kConsumers) {
         const int gq = lane >> 2, t = lane & 3;
-        const int colw = 32 * (warp & 3) + 4 * gq;
-        const int khalf = warp >> 2;
+        const int colw = 32 * warp + 4 * gq;
         const int chunk = colw >> 3;
         const uint32_t owner = static_cast<uint32_t>(chunk % p.splits);
         const int lc = (chunk / p.splits) * 8 + (colw & 7);
@@ -333,7 +387,7 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
             const int tok = 2 * t + tk;
             if (tok < p.M) {
                 const float4 v = make_float4(acc[0][tk], acc[0][2 + tk], acc[1][tk], acc[1][2 + tk]);
-                const int off = (((split * KH + khalf) * 8 + tok) * cpo + lc) * 4;
+                const int off = ((split * 8 + tok) * cpo + lc) * 4;
                 st_async_f4(map_to_rank(smem_u32(recv) + off, owner), v, rbar);
             }
         }
@@ -360,14 +414,10 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = 0.0f;
         for (int r = 0; r < p.splits; ++r) {
-#pragma unroll
-            for (int h = 0; h < KH; ++h) {
-                const float4 *src =
-                    reinterpret_cast<const float4 *>(recv + ((r * KH + h) * 8 + tok) * cpo + lch * 8);
-                const float4 lo = src[0], hi = src[1];
-                v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
-                v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
-            }
+            const float4 *src = reinterpret_cast<const float4 *>(recv + (r * 8 + tok) * cpo + lch * 8);
+            const float4 lo = src[0], hi = src[1];
+            v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+            v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
         }
         uint4 o;
         o.x = __half_as_ushort(__float2half_rn(v[0])) | (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[1]))) << 16);
@@ -379,13 +429,13 @@ __global__ void __launch_bounds__(32 * (4 * KH + 1), 1)
     cluster_wait_acquire();
 }
 
-template <int S, int KH>
+template <int S, int MT>
 cudaError_t launch_gemv_one(const GemvPlan &plan, const CUtensorMap &tmQ, const GemvParams &prm,
                             cudaStream_t st)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.splits, plan.n_tiles, 1);
-    cfg.blockDim = dim3(32 * (4 * KH + 1), 1, 1);
+    cfg.blockDim = dim3(32 * (kConsumers + 1), 1, 1);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -397,13 +447,13 @@ cudaError_t launch_gemv_one(const GemvPlan &plan, const CUtensorMap &tmQ, const 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<S, KH>, tmQ, prm);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<S, MT>, tmQ, prm);
 }
 
-template <int S, int KH>
+template <int S, int MT>
 cudaError_t configure_gemv_one()
 {
-    return cudaFuncSetAttribute(gemv_kernel<S, KH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(gemv_kernel<S, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kSmemOptIn);
 }
 
@@ -422,11 +472,10 @@ cudaError_t configure_gemv()
 
 bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
 {
-    if (M < 1 || M > 8) return false;
+    if (M < 1 || M > 2) return false;
     const int G = K / kGroup;
     const int max_split = G < 8 ? G : 8;
     pl->n_tiles = (N + kBN - 1) / kBN;
-    pl->kh = 1;
     // splits is a power of two so each cluster rank owns 128 / splits columns.
     // Measured on the decode shapes (K 4096..14336, N 4096..28672): with at
     // most one 128-column tile per SM, an 8-deep ring and the largest split
@@ -452,14 +501,14 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     // (+ 8 B per group half); find the smallest split at or above the choice that fits
     for (; splits <= max_pow2; splits *= 2) {
         const int gmax = (G + splits - 1) / splits;
-        if (static_cast<size_t>(M) * gmax * (256 + 8 * pl->kh) <= 80 * 1024) break;
+        if (static_cast<size_t>(M) * gmax * (256 + 8) <= 80 * 1024) break;
     }
     if (splits > max_pow2) return false;
     pl->splits = splits;
     const int gmax = (G + splits - 1) / splits;
     pl->xpro_bytes = M * gmax * 256;
-    pl->gmeta_bytes = (M * gmax * pl->kh * 8 + 15) & ~15;
-    pl->recv_bytes = pl->kh * 8 * kBN * 4;
+    pl->gmeta_bytes = (M * gmax * 8 + 15) & ~15;
+    pl->recv_bytes = 8 * kBN * 4;
     pl->smem = 1024 + static_cast<size_t>(pl->stages) * kStageBytes + pl->xpro_bytes + pl->gmeta_bytes +
                pl->recv_bytes + (2 * pl->stages + 1) * sizeof(uint64_t);
     return true;
@@ -488,13 +537,10 @@ cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __ha
     prm.mask_hi = 0x00F000F0u;
     prm.magic = 0x64006400u;
     if (plan.stages == 6)
-        return plan.kh == 2 ? launch_gemv_one<6, 2>(plan, tmQ, prm, st)
-                            : launch_gemv_one<6, 1>(plan, tmQ, prm, st);
+        return M == 2 ? launch_gemv_one<6, 2>(plan, tmQ, prm, st) : launch_gemv_one<6, 1>(plan, tmQ, prm, st);
     if (plan.stages == 4)
-        return plan.kh == 2 ? launch_gemv_one<4, 2>(plan, tmQ, prm, st)
-                            : launch_gemv_one<4, 1>(plan, tmQ, prm, st);
-    return plan.kh == 2 ? launch_gemv_one<8, 2>(plan, tmQ, prm, st)
-                        : launch_gemv_one<8, 1>(plan, tmQ, prm, st);
+        return M == 2 ? launch_gemv_one<4, 2>(plan, tmQ, prm, st) : launch_gemv_one<4, 1>(plan, tmQ, prm, st);
+    return M == 2 ? launch_gemv_one<8, 2>(plan, tmQ, prm, st) : launch_gemv_one<8, 1>(plan, tmQ, prm, st);
 }
 
 }  // namespace awq
