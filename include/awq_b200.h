@@ -203,7 +203,7 @@ AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s
  *   X binary16 [1, K], Y binary16 [1, N].
  * awq_w4a16_gemm takes any 1 <= M <= AWQ_MAX_M and picks its tile path
  * internally: the decode GEMV for M <= 2, register-fed tensor cores for
- * 3 <= M < 40, tcgen05/TMEM for M >= 40 (small batch from 40, prefill from 64).
+ * 3 <= M < 24, tcgen05/TMEM for M >= 24 (small batch from 24, prefill from 64).
  *   K % 128 == 0, N % 8 == 0, Q/scales/zeros as produced by awq_quantize_pack;
  *   zeros = NULL for weights from awq_quantize_pack_symmetric (zero point 8).
  *   s = NULL when X already holds X/s (1/s folded into the operator that

@@ -206,14 +206,15 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
             return AWQ_ERR_CUDA;
         return from_cuda(awq::launch_gemv(gplan, tmQ, hX, hs, hsc, zeros, hY, m, k, n, dev_status, st));
     }
-    // From about 40 tokens the small-batch layer needs more MMA rate than
-    // mma.sync gives: tcgen05 with the weights as the 128-row operand
-    // (measured on the 13B shapes: faster at 48 tokens, slower at 16 and 32).
-    if (M >= 40 && M < 64) {
+    // From about 24 tokens the small-batch layer needs more MMA rate than
+    // mma.sync gives: tcgen05 with the dequantized weights in tensor memory as
+    // the 128-row operand (measured on the 13B shapes: as fast at 24 tokens,
+    // faster from 32, slower at 8 and 16).
+    if (M >= 24 && M < 64) {
         const awq::TcsPlan plan = awq::plan_tcs(m, k, n, sms);
         if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
                        static_cast<uint32_t>(plan.nt), CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 8,
+            !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 16,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
             return AWQ_ERR_CUDA;
         e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));

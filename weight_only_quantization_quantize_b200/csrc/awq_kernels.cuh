@@ -67,7 +67,7 @@ cudaError_t launch_tct(const TctPlan &plan, const CUtensorMap &tmX, const CUtens
                        const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                        int32_t *status, cudaStream_t st);
 
-// matmul_tcs.cu -- 40 <= M < 64: tcgen05 with the weights as the 128-row operand
+// matmul_tcs.cu -- 24 <= M < 64: tcgen05 with the weights as the 128-row operand in TMEM
 struct TcsPlan {
     int nt;        // tokens padded to a multiple of 16
     int n_tiles;   // 128-column tiles

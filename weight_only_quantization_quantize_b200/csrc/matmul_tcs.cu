@@ -1,4 +1,4 @@
-// matmul_tcs.cu -- Y = (X / s) . dequant(Q) for small batches (40 <= M < 64
+// matmul_tcs.cu -- Y = (X / s) . dequant(Q) for small batches (24 <= M < 64
 // tokens) on the 5th-generation tensor cores, with the roles of the operands
 // swapped: the dequantized weights are the 128-row A operand and the tokens
 // (padded to a multiple of 16) are the N dimension.
@@ -14,19 +14,27 @@
 //
 // One CTA = 128 output columns x one k range; the k ranges of a column tile are
 // the CTAs of a thread-block cluster (split-K, up to 8):
-//   warp 0      TMA ring (4 stages): X' tile [Nt tokens x 64 k] (128-byte
-//               swizzle; tokens beyond M read as zero), packed words
-//               [8 x 128]; cp.async of the group's steps and zero words.
-//   warp 1      allocates 256 TMEM columns (four accumulators); one lane
-//               issues tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = Nt,
-//               K = 16) x 4 per stage, k-step j into accumulator j, and commits
-//               each stage back to both rings.
-//   warps 2..9  dequantize: each writes (q - z) * step for 32 columns x 32 k
-//               as binary16 into the K-major, 128-byte-swizzled A operand
-//               (4-slot ring); then read the accumulator (tcgen05.ld) and push
-//               it to the cluster CTA that owns those columns (st.async); each
-//               CTA adds the k-split partials of its columns in rank order
+//   warp 0      TMA ring (4 stages of one group, 128 k): X' tile [Nt tokens x
+//               128 k] as two 64-k chunks (128-byte swizzle; tokens beyond M
+//               read as zero), packed words [16 x 128]; cp.async of the
+//               group's steps and zero words.  One producer thread issues a
+//               stage's copies in several hundred cycles, so a stage carries a
+//               whole group.
+//   warp 1      allocates 256 TMEM columns (two accumulators and a 4-slot
+//               ring of dequantized A tiles); warps 1 and 10 each issue, from
+//               one lane, tcgen05.mma.cta_group::1.kind::f16 with A from tensor
+//               memory (M = 128, N = Nt, K = 16) x 8 per stage for every other
+//               stage into their own accumulator, and commit each stage back to
+//               both rings.
+//   warps 2..9  dequantize: warp w owns TMEM lanes 32 (w % 4) .. +31 (one
+//               output column per lane) and half of a stage's packed rows, and
+//               writes 32 columns of (q - z) * step binary16 pairs into the A
+//               slot (tcgen05.st, 2-slot ring); then read the accumulator (tcgen05.ld) and
+//               push it to the cluster CTA that owns those columns (st.async);
+//               each CTA adds the k-split partials of its columns in rank order
 //               and writes Y.
+// The dequantized weights never pass through shared memory, which then
+// carries only the TMA loads and the MMA's reads of the X' tile.
 // Within each 8-channel chunk the contraction runs in the pair order
 // (0,4),(1,5),(2,6),(3,7) on both operands (X' is stored that way by the
 // pre-pass), which leaves the sum unchanged.
@@ -37,20 +45,24 @@ namespace awq {
 namespace {
 
 constexpr int kBN = 128;               // output columns per CTA (MMA M)
-constexpr int kBK = 64;                // k per stage
+constexpr int kBK = 128;               // k per stage: one group
 constexpr int kLoadStages = 4;
-constexpr int kAStages = 4;  // dequantized A operand
+constexpr int kASlots = 2;             // dequantized A tiles in tensor memory
+constexpr int kASlotCols = kBK / 2;    // 64 TMEM columns: 128 binary16 per lane
 constexpr int kDequantWarps = 8;
-constexpr int kThreads = 64 + 32 * kDequantWarps;
-constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 4 KB of packed words
+// Two MMA issuers (warps 1 and 2 + kDequantWarps), each with its own
+// accumulator and every other stage: one thread issues a tcgen05.mma only every
+// ~140 cycles whatever N is, so at a few dozen tokens the issue rate, not the
+// tensor core, bounds the stream.  The accumulators are added in the epilogue.
+constexpr int kIssuers = 2;
+constexpr int kIssuer2Warp = 2 + kDequantWarps;
+constexpr int kThreads = 32 * (3 + kDequantWarps);
+constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 8 KB of packed words
 constexpr int kMetaBytes = 1024;              // 256 B steps + 64 B zero words, padded
-constexpr int kABytes = kBN * kBK * 2;        // 16 KB
-// Four accumulators of up to 64 token columns: k-step j of every stage adds
-// into accumulator j, so four independent tcgen05.mma chains are in flight
-// instead of one; the epilogue adds them in the fixed order 0, 1, 2, 3.
-constexpr int kAccs = kBK / 16;
-constexpr int kAccCols = 64;
-constexpr int kTmemCols = kAccs * kAccCols;
+constexpr int kAccCols = 64;                  // an accumulator: up to 64 token columns
+constexpr int kACol = kIssuers * kAccCols;    // A slots after the accumulators
+constexpr int kTmemCols = 256;                // two CTAs per SM share the 512 columns
+constexpr size_t kMinSmem = 80 * 1024;        // limits residency to two CTAs per SM
 
 struct Params {
     const __half *scales;
@@ -76,13 +88,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *smem = align1024(smem_dyn);
-    uint8_t *aring = smem + kLoadStages * p.stage_bytes;  // 1 KB aligned
-    uint64_t *full_load = reinterpret_cast<uint64_t *>(aring + kAStages * kABytes);
+    uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + kLoadStages * p.stage_bytes);
     uint64_t *empty_load = full_load + kLoadStages;
     uint64_t *full_a = empty_load + kLoadStages;
-    uint64_t *empty_a = full_a + kAStages;
-    uint64_t *tmem_full = empty_a + kAStages;
-    uint64_t *recv_bar = tmem_full + 1;
+    uint64_t *empty_a = full_a + kASlots;
+    uint64_t *tmem_full = empty_a + kASlots;  // one per issuer
+    uint64_t *recv_bar = tmem_full + kIssuers;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(recv_bar + 1);
     // after the main loop the load ring is idle: it receives the pushed partials
     float *recv = reinterpret_cast<float *>(smem);
@@ -96,7 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * KB / p.splits);
     const int nkb = kb_end - kb_begin;
     const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
-    const int xbytes = p.nt * 128;
+    const int xchunk = p.nt * 128;  // one 64-k chunk of the X' tile (a 128-byte swizzle atom wide)
+    const int xbytes = 2 * xchunk;
 
     pdl_launch_dependents();
 
@@ -105,11 +117,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full_load[i], 1 + 32);  // expect_tx + 32 cp.async arrivals
             mbar_init(&empty_load[i], 1);      // MMA commit
         }
-        for (int i = 0; i < kAStages; ++i) {
+        for (int i = 0; i < kASlots; ++i) {
             mbar_init(&full_a[i], kDequantWarps);
             mbar_init(&empty_a[i], 1);         // MMA commit
         }
-        mbar_init(tmem_full, 1);
+        for (int i = 0; i < kIssuers; ++i) mbar_init(&tmem_full[i], 1);
         mbar_init(recv_bar, 1);
         fence_barrier_init();
         mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(p.splits * p.nt * cpo * 4));
@@ -145,10 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 mbar_arrive_expect_tx(&full_load[st], static_cast<uint32_t>(xbytes + kQBytes));
                 tma_load_2d(stg, &tmX, &full_load[st], kb * kBK, 0);
+                tma_load_2d(stg + xchunk, &tmX, &full_load[st], kb * kBK + 64, 0);
                 tma_load_2d(stg + xbytes, &tmQ, &full_load[st], n0, kb * (kBK / 8));
             }
             uint8_t *meta = stg + xbytes + kQBytes;
-            const int g = (kb * kBK) / kGroup;
+            const int g = kb;  // one group per stage
             if (lane < 16) {
                 const int n = n0 + 8 * lane;
                 const bool in = n < p.N;
@@ -164,75 +177,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == kIssuer2Warp) {
+        // ------------------------------------------------------------ MMA issuers
+        const int issuer = warp == 1 ? 0 : 1;
+        const uint32_t acc_d = tmem_base + issuer * kAccCols;
         const uint32_t idesc = tc_idesc_f16(kBN, p.nt);
-        for (int i = 0; i < nkb; ++i) {
+        for (int i = issuer; i < nkb; i += kIssuers) {
             const int st = i % kLoadStages;
-            const int as = i % kAStages;
-            if (!mbar_wait(&full_load[st], (i / kLoadStages) & 1) || !mbar_wait(&full_a[as], (i / kAStages) & 1)) {
+            const int as = i % kASlots;
+            // the outcome is voted so that the warp leaves the loop as one
+            bool w = mbar_wait(&full_load[st], (i / kLoadStages) & 1);
+            if (w) w = mbar_wait(&full_a[as], (i / kASlots) & 1);
+            if (!__all_sync(0xffffffffu, w)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t a0 = smem_u32(aring + as * kABytes);
+                const uint32_t a0 = tmem_base + kACol + as * kASlotCols;
                 const uint32_t b0 = smem_u32(smem + st * p.stage_bytes);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
-                    tc_mma(tmem_base + k * kAccCols, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), idesc,
-                           i > 0 ? 1u : 0u);
+                    tc_mma_ta(acc_d, a0 + 8 * k, sw128_desc(b0 + (k >> 2) * xchunk + 32 * (k & 3)), idesc,
+                              (i > issuer || k > 0) ? 1u : 0u);
                 tc_commit(&empty_load[st]);
                 tc_commit(&empty_a[as]);
             }
             __syncwarp();
         }
         if (lane == 0) {
-            if (ok)
-                tc_commit(tmem_full);
-            else
+            // tmem_full completes once every MMA issued has completed; after a
+            // timeout this lane waits for that itself before TMEM is freed
+            tc_commit(&tmem_full[issuer]);
+            if (!ok) {
                 report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+                mbar_wait_for(&tmem_full[issuer], 0, kDrainLimitNs);
+            }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ dequant
-        // warp d: column 32 * (d % 4) + lane, packed rows 4 * (d / 4) .. +3 of the stage
-        const int dw = warp - 2;
-        const int c = 32 * (dw & 3) + lane;
-        const int r0 = 4 * (dw >> 2);
+        // warp w: TMEM lanes 32 (w % 4) .. +31 = output columns; packed rows
+        // 4 h .. 4 h + 3 of each stage (h = 0 for warps 2..5, 1 for 6..9)
+        const int quarter = warp & 3;
+        const int h = (warp - 2) >> 2;
+        const int c = 32 * quarter + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const UnpackConsts uk = p.uk;
         for (int i = 0; i < nkb; ++i) {
             const int st = i % kLoadStages;
-            const int as = i % kAStages;
-            if (!mbar_wait(&full_load[st], (i / kLoadStages) & 1) ||
-                (i >= kAStages && !mbar_wait(&empty_a[as], ((i / kAStages) - 1) & 1))) {
+            const int as = i % kASlots;
+            bool w = mbar_wait(&full_load[st], (i / kLoadStages) & 1);
+            if (w && i >= kASlots) w = mbar_wait(&empty_a[as], ((i / kASlots) - 1) & 1);
+            if (!__all_sync(0xffffffffu, w)) {
                 ok = false;
                 break;
             }
+            tc_fence_after();
             const uint8_t *q = smem + st * p.stage_bytes + xbytes;
             const uint8_t *meta = q + kQBytes;
-            const uint32_t abase = smem_u32(aring + as * kABytes);
             const uint16_t sbits = reinterpret_cast<const uint16_t *>(meta)[c];
             const uint32_t sc2 = static_cast<uint32_t>(sbits) | (static_cast<uint32_t>(sbits) << 16);
             const uint32_t zw = reinterpret_cast<const uint32_t *>(meta + 256)[c >> 3];
             uint32_t za, zb;
             zero_constants((zw >> (4 * (c & 7))) & 15u, za, zb);
-            uint32_t w[4];
+            uint32_t wv[8];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) w[r] = reinterpret_cast<const uint32_t *>(q + (r0 + r) * (kBN * 4))[c];
+            for (int r = 0; r < 8; ++r) wv[r] = reinterpret_cast<const uint32_t *>(q + (8 * h + r) * (kBN * 4))[c];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                uint32_t d[4];
-                unpack_minus_zero(w[r], za, zb, d, uk);
-                uint32_t o[4];
+            for (int part = 0; part < 2; ++part) {
+                uint32_t o[16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[j]) : "r"(d[j]), "r"(sc2));
-                const uint32_t dst = abase + c * 128 + (((r0 + r) ^ (c & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
-                             "r"(o[2]), "r"(o[3])
-                             : "memory");
+                for (int r = 0; r < 4; ++r) {
+                    uint32_t d[4];
+                    unpack_minus_zero(wv[4 * part + r], za, zb, d, uk);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[4 * r + j]) : "r"(d[j]), "r"(sc2));
+                }
+                tmem_st16(tmem_base + lane_addr + kACol + as * kASlotCols + 32 * h + 16 * part, o);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&full_a[as]);
         }
@@ -244,13 +270,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32 (w % 4) .. +31 (output columns) and takes half of the token columns.
     // Every partial goes to the cluster rank owning its column: rank c / cpo,
     // laid out there as [source rank][token][owned column].
-    const bool have_acc = warp >= 2 && ok && mbar_wait(tmem_full, 0);
-    if (warp >= 2 && !have_acc && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
+    const bool dq = warp >= 2 && warp < kIssuer2Warp;  // a dequantization warp
+    const bool have_acc =
+        dq && __all_sync(0xffffffffu, ok && mbar_wait(&tmem_full[0], 0) && mbar_wait(&tmem_full[1], 0));
+    const bool two = nkb >= 2;  // with one stage the second accumulator holds nothing
+    if (dq && !have_acc && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     // Every CTA of the cluster is past its main loop (its load ring, which
     // receives the partials, is idle) and has initialized its barriers.
     cluster_arrive_release();
     cluster_wait_acquire();
-    if (warp >= 2) {
+    if (dq) {
         tc_fence_after();
         const int quarter = warp & 3;
         const int col = quarter * 32 + lane;
@@ -261,17 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
         const uint32_t rbase = map_to_rank(smem_u32(recv), owner);
         for (int t0 = tb; t0 < tb + p.nt / 2; t0 += 8) {
-            float sum[8];
-#pragma unroll
-            for (int a = 0; a < kAccs; ++a) {
-                uint32_t v[8];
-                tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * kAccCols + t0, v);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) sum[j] = a == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
-            }
+            uint32_t v[8], v1[8];
+            tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + t0, v);
+            tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kAccCols + t0, v1);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float x = have_acc ? sum[j] : 0.0f;
+                const float x = have_acc ? __uint_as_float(v[j]) + (two ? __uint_as_float(v1[j]) : 0.0f) : 0.0f;
                 const int off = ((split * p.nt + t0 + j) * cpo + lc) * 4;
                 st_async_f32(rbase + off, x, rbar);
             }
@@ -314,9 +338,12 @@ TcsPlan plan_tcs(int M, int K, int N, int num_sms)
     int splits = 1;
     while (splits * 2 <= 8 && pl.n_tiles * splits * 2 <= 2 * num_sms && KB / (splits * 2) >= 4) splits *= 2;
     pl.splits = splits;
-    pl.stage_bytes = pl.nt * 128 + kQBytes + kMetaBytes;
-    pl.smem = 1024 + static_cast<size_t>(kLoadStages) * pl.stage_bytes + static_cast<size_t>(kAStages) * kABytes +
-              256;
+    pl.stage_bytes = 2 * pl.nt * 128 + kQBytes + kMetaBytes;
+    pl.smem = 1024 + static_cast<size_t>(kLoadStages) * pl.stage_bytes + 256;
+    // At most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns,
+    // and a third would block in tcgen05.alloc while its cluster peers wait
+    // for it.  The shared-memory request enforces that.
+    if (pl.smem < kMinSmem) pl.smem = kMinSmem;
     return pl;
 }
 
