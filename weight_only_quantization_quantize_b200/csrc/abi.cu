@@ -214,7 +214,7 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         const awq::TcsPlan plan = awq::plan_tcs(m, k, n, sms);
         if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
                        static_cast<uint32_t>(plan.nt), CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 16,
+            !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 8,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
             return AWQ_ERR_CUDA;
         e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));

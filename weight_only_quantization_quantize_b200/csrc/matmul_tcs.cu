@@ -14,22 +14,17 @@
 //
 // One CTA = 128 output columns x one k range; the k ranges of a column tile are
 // the CTAs of a thread-block cluster (split-K, up to 8):
-//   warp 0      TMA ring (4 stages of one group, 128 k): X' tile [Nt tokens x
-//               128 k] as two 64-k chunks (128-byte swizzle; tokens beyond M
-//               read as zero), packed words [16 x 128]; cp.async of the
-//               group's steps and zero words.  One producer thread issues a
-//               stage's copies in several hundred cycles, so a stage carries a
-//               whole group.
-//   warp 1      allocates 256 TMEM columns (two accumulators and a 4-slot
-//               ring of dequantized A tiles); warps 1 and 10 each issue, from
-//               one lane, tcgen05.mma.cta_group::1.kind::f16 with A from tensor
-//               memory (M = 128, N = Nt, K = 16) x 8 per stage for every other
-//               stage into their own accumulator, and commit each stage back to
-//               both rings.
-//   warps 2..9  dequantize: warp w owns TMEM lanes 32 (w % 4) .. +31 (one
-//               output column per lane) and half of a stage's packed rows, and
-//               writes 32 columns of (q - z) * step binary16 pairs into the A
-//               slot (tcgen05.st, 2-slot ring); then read the accumulator (tcgen05.ld) and
+//   warp 0      TMA ring (4 stages): X' tile [Nt tokens x 64 k] (128-byte
+//               swizzle; tokens beyond M read as zero), packed words [8 x 128];
+//               cp.async of the group's steps and zero words.
+//   warp 1      allocates 128 TMEM columns (the accumulator and a 2-slot ring
+//               of dequantized A tiles); one lane issues
+//               tcgen05.mma.cta_group::1.kind::f16 with A from tensor memory
+//               (M = 128, N = Nt, K = 16) x 4 per stage and commits each stage
+//               back to both rings.
+//   warps 2..5  dequantize: warp w owns TMEM lanes 32 (w % 4) .. +31 (one
+//               output column per lane) and writes the stage's 32 columns of
+//               (q - z) * step binary16 pairs into the A slot (tcgen05.st); then read the accumulator (tcgen05.ld) and
 //               push it to the cluster CTA that owns those columns (st.async);
 //               each CTA adds the k-split partials of its columns in rank order
 //               and writes Y.
@@ -45,24 +40,23 @@ namespace awq {
 namespace {
 
 constexpr int kBN = 128;               // output columns per CTA (MMA M)
-constexpr int kBK = 128;               // k per stage: one group
+constexpr int kBK = 64;                // k per stage
 constexpr int kLoadStages = 4;
 constexpr int kASlots = 2;             // dequantized A tiles in tensor memory
-constexpr int kASlotCols = kBK / 2;    // 64 TMEM columns: 128 binary16 per lane
-constexpr int kDequantWarps = 8;
-// Two MMA issuers (warps 1 and 2 + kDequantWarps), each with its own
-// accumulator and every other stage: one thread issues a tcgen05.mma only every
-// ~140 cycles whatever N is, so at a few dozen tokens the issue rate, not the
-// tensor core, bounds the stream.  The accumulators are added in the epilogue.
-constexpr int kIssuers = 2;
-constexpr int kIssuer2Warp = 2 + kDequantWarps;
-constexpr int kThreads = 32 * (3 + kDequantWarps);
-constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 8 KB of packed words
+constexpr int kASlotCols = kBK / 2;    // 32 TMEM columns: 64 binary16 per lane
+constexpr int kDequantWarps = 4;
+// A CTA issues one tcgen05.mma (1 KB of packed weights at M = 128, K = 16)
+// every ~140 cycles whatever N is, so at a few dozen tokens the MMA issue rate
+// of a CTA, not the tensor core, bounds its stream: four small CTAs per SM.
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+constexpr int kQBytes = (kBK / 8) * kBN * 4;  // 4 KB of packed words
 constexpr int kMetaBytes = 1024;              // 256 B steps + 64 B zero words, padded
-constexpr int kAccCols = 64;                  // an accumulator: up to 64 token columns
-constexpr int kACol = kIssuers * kAccCols;    // A slots after the accumulators
-constexpr int kTmemCols = 256;                // two CTAs per SM share the 512 columns
-constexpr size_t kMinSmem = 80 * 1024;        // limits residency to two CTAs per SM
+constexpr int kAccCols = 64;                  // the accumulator: up to 64 token columns
+constexpr int kACol = kAccCols;               // A slots after the accumulator
+constexpr int kTmemCols = 128;                // four CTAs per SM share the 512 columns
+constexpr int kCtasPerSm = 4;
+constexpr size_t kSmemPerSm = 233472;         // shared memory of an SM
+constexpr size_t kMinSmem = kSmemPerSm / (kCtasPerSm + 1) + 1024;  // a fifth CTA never fits
 
 struct Params {
     const __half *scales;
@@ -92,8 +86,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *empty_load = full_load + kLoadStages;
     uint64_t *full_a = empty_load + kLoadStages;
     uint64_t *empty_a = full_a + kASlots;
-    uint64_t *tmem_full = empty_a + kASlots;  // one per issuer
-    uint64_t *recv_bar = tmem_full + kIssuers;
+    uint64_t *tmem_full = empty_a + kASlots;
+    uint64_t *recv_bar = tmem_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(recv_bar + 1);
     // after the main loop the load ring is idle: it receives the pushed partials
     float *recv = reinterpret_cast<float *>(smem);
@@ -107,8 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * KB / p.splits);
     const int nkb = kb_end - kb_begin;
     const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
-    const int xchunk = p.nt * 128;  // one 64-k chunk of the X' tile (a 128-byte swizzle atom wide)
-    const int xbytes = 2 * xchunk;
+    const int xbytes = p.nt * 128;
 
     pdl_launch_dependents();
 
@@ -121,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full_a[i], kDequantWarps);
             mbar_init(&empty_a[i], 1);         // MMA commit
         }
-        for (int i = 0; i < kIssuers; ++i) mbar_init(&tmem_full[i], 1);
+        mbar_init(tmem_full, 1);
         mbar_init(recv_bar, 1);
         fence_barrier_init();
         mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(p.splits * p.nt * cpo * 4));
@@ -157,11 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 mbar_arrive_expect_tx(&full_load[st], static_cast<uint32_t>(xbytes + kQBytes));
                 tma_load_2d(stg, &tmX, &full_load[st], kb * kBK, 0);
-                tma_load_2d(stg + xchunk, &tmX, &full_load[st], kb * kBK + 64, 0);
                 tma_load_2d(stg + xbytes, &tmQ, &full_load[st], n0, kb * (kBK / 8));
             }
             uint8_t *meta = stg + xbytes + kQBytes;
-            const int g = kb;  // one group per stage
+            const int g = (kb * kBK) / kGroup;
             if (lane < 16) {
                 const int n = n0 + 8 * lane;
                 const bool in = n < p.N;
@@ -177,12 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
-    } else if (warp == 1 || warp == kIssuer2Warp) {
-        // ------------------------------------------------------------ MMA issuers
-        const int issuer = warp == 1 ? 0 : 1;
-        const uint32_t acc_d = tmem_base + issuer * kAccCols;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
         const uint32_t idesc = tc_idesc_f16(kBN, p.nt);
-        for (int i = issuer; i < nkb; i += kIssuers) {
+        for (int i = 0; i < nkb; ++i) {
             const int st = i % kLoadStages;
             const int as = i % kASlots;
             // the outcome is voted so that the warp leaves the loop as one
@@ -198,8 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b0 = smem_u32(smem + st * p.stage_bytes);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
-                    tc_mma_ta(acc_d, a0 + 8 * k, sw128_desc(b0 + (k >> 2) * xchunk + 32 * (k & 3)), idesc,
-                              (i > issuer || k > 0) ? 1u : 0u);
+                    tc_mma_ta(tmem_base, a0 + 8 * k, sw128_desc(b0 + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
                 tc_commit(&empty_load[st]);
                 tc_commit(&empty_a[as]);
             }
@@ -208,19 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // tmem_full completes once every MMA issued has completed; after a
             // timeout this lane waits for that itself before TMEM is freed
-            tc_commit(&tmem_full[issuer]);
+            tc_commit(tmem_full);
             if (!ok) {
                 report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
-                mbar_wait_for(&tmem_full[issuer], 0, kDrainLimitNs);
+                mbar_wait_for(tmem_full, 0, kDrainLimitNs);
             }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ dequant
-        // warp w: TMEM lanes 32 (w % 4) .. +31 = output columns; packed rows
-        // 4 h .. 4 h + 3 of each stage (h = 0 for warps 2..5, 1 for 6..9)
+        // warp w: TMEM lanes 32 (w % 4) .. +31 = output columns, every packed
+        // row of the stage
         const int quarter = warp & 3;
-        const int h = (warp - 2) >> 2;
         const int c = 32 * quarter + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const UnpackConsts uk = p.uk;
@@ -243,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             zero_constants((zw >> (4 * (c & 7))) & 15u, za, zb);
             uint32_t wv[8];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) wv[r] = reinterpret_cast<const uint32_t *>(q + (8 * h + r) * (kBN * 4))[c];
+            for (int r = 0; r < 8; ++r) wv[r] = reinterpret_cast<const uint32_t *>(q + r * (kBN * 4))[c];
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 uint32_t o[16];
@@ -255,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 4; ++j)
                         asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[4 * r + j]) : "r"(d[j]), "r"(sc2));
                 }
-                tmem_st16(tmem_base + lane_addr + kACol + as * kASlotCols + 32 * h + 16 * part, o);
+                tmem_st16(tmem_base + lane_addr + kACol + as * kASlotCols + 16 * part, o);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -267,13 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- epilogue
     // Dequant warps read the accumulator: warp w reaches TMEM lanes
-    // 32 (w % 4) .. +31 (output columns) and takes half of the token columns.
+    // 32 (w % 4) .. +31 (output columns), every token column.
     // Every partial goes to the cluster rank owning its column: rank c / cpo,
     // laid out there as [source rank][token][owned column].
-    const bool dq = warp >= 2 && warp < kIssuer2Warp;  // a dequantization warp
-    const bool have_acc =
-        dq && __all_sync(0xffffffffu, ok && mbar_wait(&tmem_full[0], 0) && mbar_wait(&tmem_full[1], 0));
-    const bool two = nkb >= 2;  // with one stage the second accumulator holds nothing
+    const bool dq = warp >= 2;  // a dequantization warp
+    const bool have_acc = dq && __all_sync(0xffffffffu, ok && mbar_wait(tmem_full, 0));
     if (dq && !have_acc && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     // Every CTA of the cluster is past its main loop (its load ring, which
     // receives the partials, is idle) and has initialized its barriers.
@@ -283,19 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int quarter = warp & 3;
         const int col = quarter * 32 + lane;
-        const int half = (warp - 2) >> 2;
-        const int tb = half * (p.nt / 2);
         const uint32_t owner = static_cast<uint32_t>(col / cpo);
         const int lc = col - static_cast<int>(owner) * cpo;
         const uint32_t rbar = map_to_rank(smem_u32(recv_bar), owner);
         const uint32_t rbase = map_to_rank(smem_u32(recv), owner);
-        for (int t0 = tb; t0 < tb + p.nt / 2; t0 += 8) {
-            uint32_t v[8], v1[8];
+        for (int t0 = 0; t0 < p.nt; t0 += 8) {
+            uint32_t v[8];
             tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + t0, v);
-            tmem_ld8(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kAccCols + t0, v1);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float x = have_acc ? __uint_as_float(v[j]) + (two ? __uint_as_float(v1[j]) : 0.0f) : 0.0f;
+                const float x = have_acc ? __uint_as_float(v[j]) : 0.0f;
                 const int off = ((split * p.nt + t0 + j) * cpo + lc) * 4;
                 st_async_f32(rbase + off, x, rbar);
             }
@@ -333,15 +316,16 @@ TcsPlan plan_tcs(int M, int K, int N, int num_sms)
     pl.nt = (M + 15) / 16 * 16;
     pl.n_tiles = (N + kBN - 1) / kBN;
     const int KB = K / kBK;
-    // Two CTAs per SM fit; the largest power-of-two split that keeps one wave
+    // Four CTAs per SM fit; the largest power-of-two split that keeps one wave
     // and leaves every CTA at least four stages.
     int splits = 1;
-    while (splits * 2 <= 8 && pl.n_tiles * splits * 2 <= 2 * num_sms && KB / (splits * 2) >= 4) splits *= 2;
+    while (splits * 2 <= 8 && pl.n_tiles * splits * 2 <= kCtasPerSm * num_sms && KB / (splits * 2) >= 4)
+        splits *= 2;
     pl.splits = splits;
-    pl.stage_bytes = 2 * pl.nt * 128 + kQBytes + kMetaBytes;
+    pl.stage_bytes = pl.nt * 128 + kQBytes + kMetaBytes;
     pl.smem = 1024 + static_cast<size_t>(kLoadStages) * pl.stage_bytes + 256;
-    // At most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns,
-    // and a third would block in tcgen05.alloc while its cluster peers wait
+    // At most four CTAs per SM: each holds 128 of the SM's 512 TMEM columns,
+    // and a fifth would block in tcgen05.alloc while its cluster peers wait
     // for it.  The shared-memory request enforces that.
     if (pl.smem < kMinSmem) pl.smem = kMinSmem;
     return pl;
