@@ -103,6 +103,11 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.xpro_bytes + p.gmeta_bytes + p.recv_bytes);
     uint64_t *empty = full + S;
     uint64_t *recv_bar = empty + S;
+    // 256 zero bytes: the B operand of lanes whose token column is not the
+    // stage's group reads them (one address select per stage, no per-load
+    // predication)
+    uint8_t *zchunk = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(recv_bar + 1) + 15) & ~uintptr_t(15));
+    if (threadIdx.x < 64) reinterpret_cast<uint32_t *>(zchunk)[threadIdx.x] = 0u;
     const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
 
     if (threadIdx.x == 0) {
@@ -257,7 +262,19 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
         const int b_tok = gq % MT;
         // This lane's X' row.  A chunk index it * 16 + r XOR-swizzled by the
         // token (< 8) equals it * 16 + (r ^ token).
-        const uint8_t *xrow = xpro + static_cast<size_t>(b_tok) * chunks * 16;
+        const uint32_t xrow = smem_u32(xpro) + static_cast<uint32_t>(b_tok * chunks * 16);
+        const uint32_t zrow = smem_u32(zchunk);
+        const uint32_t qwarp = smem_u32(smem) + static_cast<uint32_t>(warp * 2048);
+        // this lane's shared-memory offsets of its four 16-byte loads per stage:
+        // packed row r = 8 (ss / 2) + 2 t + ss % 2, chunk gq XOR-swizzled by the
+        // row (128-byte TMA swizzle); X' chunk r XOR-swizzled by the token
+        uint32_t offq[4], offx[4];
+#pragma unroll
+        for (int ss = 0; ss < 4; ++ss) {
+            const int r = 8 * (ss >> 1) + 2 * t + (ss & 1);
+            offq[ss] = static_cast<uint32_t>(r * 128 + ((gq ^ (r & 7)) << 4));
+            offx[ss] = static_cast<uint32_t>((r ^ b_tok) << 4);
+        }
         const uint32_t mlo = p.mask_lo, mhi = p.mask_hi, magic = p.magic;
         float R[2][4];  // [tile][fragment element], one batch of groups
 #pragma unroll
@@ -270,16 +287,16 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
         uint2 cap_sc0 = make_uint2(0u, 0u), cap_sc1 = cap_sc0;
         uint32_t cap_z0 = 0u, cap_z1 = 0u;
         bool ok = true;
+        int st = 0;          // ring slot of the stage
+        uint32_t ph = 0;     // its phase parity
+        int j = 0;           // group within the batch
         for (int it = 0; it < ng; ++it) {
-            const int st = it % S;
-            const int j = it % kGPB;  // group within the batch
             // the outcome is voted so that the warp leaves the loop as one
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (it / S) & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph))) {
                 ok = false;
                 break;
             }
-            const uint8_t *stg = smem + st * kStageBytes;
-            const uint8_t *meta = stg + kQStage;
+            const uint8_t *meta = smem + st * kStageBytes + kQStage;
             if (t == j / kLG) {
                 const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
                 const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
@@ -289,15 +306,17 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
                 cap_sc1 = second ? sc : cap_sc1;
                 cap_z1 = second ? zw : cap_z1;
             }
-            const bool mine = b_group == j;
-            const uint8_t *qslab = stg + warp * 2048;
+            const uint32_t qbase = qwarp + static_cast<uint32_t>(st * kStageBytes);
+            const uint32_t xbase = b_group == j ? xrow + static_cast<uint32_t>(it * 256) : zrow;
 #pragma unroll
             for (int ss = 0; ss < 4; ++ss) {
-                const int r = 8 * (ss >> 1) + 2 * t + (ss & 1);
-                const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
-                uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-                if (mine) bx = *reinterpret_cast<const uint4 *>(xrow + it * 256 + ((r ^ b_tok) << 4));
-                const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+                uint32_t w[4], bx[4];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                             : "r"(qbase + offq[ss]));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(bx[0]), "=r"(bx[1]), "=r"(bx[2]), "=r"(bx[3])
+                             : "r"(xbase + offx[ss]));
                 uint32_t ev0[4], ev2[4], od1[4], od3[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -312,8 +331,8 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
                     const int c0 = 2 * tile, c1 = 2 * tile + 1;
                     const uint32_t ae[4] = {ev0[c0], ev0[c1], ev2[c0], ev2[c1]};
                     const uint32_t ao[4] = {od1[c0], od1[c1], od3[c0], od3[c1]};
-                    mma_16816(R[tile], ae, bx.x, bx.y);
-                    mma_16816(R[tile], ao, bx.z, bx.w);  // X' / 16 on the odd form
+                    mma_16816(R[tile], ae, bx[0], bx[1]);
+                    mma_16816(R[tile], ao, bx[2], bx[3]);  // X' / 16 on the odd form
                 }
             }
             __syncwarp();
@@ -356,6 +375,13 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
                 for (int a = 0; a < 2; ++a)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) R[a][i] = 0.0f;
+                j = 0;
+            } else {
+                ++j;
+            }
+            if (++st == S) {
+                st = 0;
+                ph ^= 1u;
             }
         }
         // Sum the lanes' group partials (fixed butterfly order): lane t = 0 of
@@ -510,7 +536,7 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     pl->gmeta_bytes = (M * gmax * 8 + 15) & ~15;
     pl->recv_bytes = 8 * kBN * 4;
     pl->smem = 1024 + static_cast<size_t>(pl->stages) * kStageBytes + pl->xpro_bytes + pl->gmeta_bytes +
-               pl->recv_bytes + (2 * pl->stages + 1) * sizeof(uint64_t);
+               pl->recv_bytes + (2 * pl->stages + 1) * sizeof(uint64_t) + 16 + 256;  // + zero chunk
     return true;
 }
 
