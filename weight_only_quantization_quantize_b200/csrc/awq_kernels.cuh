@@ -26,6 +26,7 @@ struct GemvPlan {
     int stages;
     int xpro_bytes;
     int gmeta_bytes;
+    int cmeta_bytes;  // the CTA's steps and zero words
     int recv_bytes;
     size_t smem;
 };

@@ -24,9 +24,10 @@
 // step / zero point arithmetic runs once per batch instead of once per group.
 //
 // Structure (one CTA = 128 output columns x a k range; clusters split K):
-//   producer warp   TMA ring of 128-row groups (four 16 x 32-word boxes,
-//                   128-byte swizzle) + cp.async of the group's steps and zero
-//                   words; ring depth 8, 6 or 4 (see plan_gemv).
+//   producer warp   cp.async of the steps and zero words of all of the CTA's
+//                   groups (once), then a TMA ring of 128-row groups (four
+//                   16 x 32-word boxes, 128-byte swizzle); ring depth 8, 6 or 4
+//                   (see plan_gemv).
 //   4 consumers     32 columns per warp; a lane turns one 16-byte load
 //                   (4 columns x 8 k) into four even-form and four odd-form
 //                   f16x2 operands with LOP3 only and feeds mma.sync.
@@ -41,8 +42,8 @@ namespace awq {
 namespace {
 
 constexpr int kBN = 128;
-constexpr int kQStage = 4 * 2048;
-constexpr int kStageBytes = 9216;  // 8 KB words + 256 B steps + 64 B zero words, padded
+constexpr int kQStage = 4 * 2048;  // one unit: 16 packed rows x 128 columns
+constexpr int kStageBytes = kQStage;
 constexpr int kSmemOptIn = 232448;
 constexpr int kConsumers = 4;  // one warp per 32-column slab of the 128-column tile
 
@@ -56,6 +57,7 @@ struct GemvParams {
     int M, K, N, G, splits;
     int xpro_bytes;   // X' buffer: M * chunks * 16
     int gmeta_bytes;  // per (token, group, half): {1024 S0 + 64 S1, S0 + S1}
+    int cmeta_bytes;  // the CTA's steps [group][128] binary16, then zero words [group][16]
     int recv_bytes;   // partials pushed to this CTA: [src rank][k half][8 tokens][128 / splits]
     // Unpack constants, passed at run time: as compile-time literals the
     // compiler re-materializes them before every use (a LOP3 encodes only one
@@ -81,7 +83,6 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
     // within a batch of kGPB groups) + token, so one accumulator fragment holds
     // kGPB groups' sums and the step / zero point are applied once per batch.
     constexpr int kGPB = 8 / MT;
-    constexpr int kLG = 2 / MT;  // groups among a lane's two fragment columns
     static_assert(MT == 1 || MT == 2, "the decode GEMV takes one or two tokens");
 
     extern __shared__ uint8_t smem_dyn[];
@@ -99,23 +100,27 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
 
     uint8_t *xpro = smem + S * kStageBytes;
     float2 *gmeta = reinterpret_cast<float2 *>(xpro + p.xpro_bytes);
-    float *recv = reinterpret_cast<float *>(xpro + p.xpro_bytes + p.gmeta_bytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(xpro + p.xpro_bytes + p.gmeta_bytes + p.recv_bytes);
+    uint8_t *csteps = xpro + p.xpro_bytes + p.gmeta_bytes;
+    uint8_t *czeros = csteps + ng * 256;
+    float *recv = reinterpret_cast<float *>(csteps + p.cmeta_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(csteps + p.cmeta_bytes + p.recv_bytes);
     uint64_t *empty = full + S;
     uint64_t *recv_bar = empty + S;
+    uint64_t *meta_bar = recv_bar + 1;  // the CTA's steps and zero words have landed
     // 256 zero bytes: the B operand of lanes whose token column is not the
     // stage's group reads them (one address select per stage, no per-load
     // predication)
-    uint8_t *zchunk = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(recv_bar + 1) + 15) & ~uintptr_t(15));
+    uint8_t *zchunk = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(meta_bar + 1) + 15) & ~uintptr_t(15));
     if (threadIdx.x < 64) reinterpret_cast<uint32_t *>(zchunk)[threadIdx.x] = 0u;
     const int cpo = kBN / p.splits;  // columns each cluster rank owns in the epilogue
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1 + 32);
+            mbar_init(&full[i], 1);
             mbar_init(&empty[i], kConsumers);
         }
         mbar_init(recv_bar, 1);
+        mbar_init(meta_bar, 32);
         fence_barrier_init();
         // expect every rank's partials for the columns this CTA owns
         mbar_arrive_expect_tx(recv_bar, MT * cpo * p.splits * 4);
@@ -153,24 +158,28 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
             uint8_t *stg = smem + st * kStageBytes;
             const int g = g_begin + it;
             if (lane == 0) {
+                // four 16 x 32-word boxes (one per consumer warp's slab), 128-byte swizzle
                 mbar_arrive_expect_tx(&full[st], kQStage);
 #pragma unroll
-                for (int w = 0; w < 4; ++w)
-                    tma_load_2d(stg + w * 2048, &tmQ, &full[st], n0 + 32 * w, g * 16);
+                for (int w = 0; w < 4; ++w) tma_load_2d(stg + w * 2048, &tmQ, &full[st], n0 + 32 * w, g * 16);
             }
-            uint8_t *meta = stg + kQStage;
-            if (lane < 16) {
-                const int n = n0 + 8 * lane;
-                const bool in = n < p.N;
-                cp_async_16(meta + 16 * lane, p.scales + static_cast<size_t>(g) * p.N + (in ? n : 0),
-                            in ? 16u : 0u);
-            } else {
-                const int wi = n0 / 8 + (lane - 16);
-                const bool in = wi < p.N / 8;
-                cp_async_4(meta + 256 + 4 * (lane - 16),
-                           zero_word_src(p.zeros, g, p.N / 8, in ? wi : 0, lane), in ? 4u : 0u);
+            if (it == pre - 1) {
+                // The steps and zero words of all of the CTA's groups, once,
+                // behind the first ring's worth of packed words.
+                for (int c = lane; c < ng * 16; c += 32) {
+                    const int gi = c >> 4, c16 = c & 15;
+                    const int gg = g_begin + gi;
+                    const int n = n0 + 8 * c16;
+                    const bool in_s = n < p.N;
+                    cp_async_16(csteps + gi * 256 + 16 * c16,
+                                p.scales + static_cast<size_t>(gg) * p.N + (in_s ? n : 0), in_s ? 16u : 0u);
+                    const int wi = n0 / 8 + c16;
+                    const bool in_z = wi < p.N / 8;
+                    cp_async_4(czeros + gi * 64 + 4 * c16, zero_word_src(p.zeros, gg, p.N / 8, in_z ? wi : 0, c16),
+                               in_z ? 4u : 0u);
+                }
+                cp_async_arrive_noinc(meta_bar);
             }
-            cp_async_arrive_noinc(&full[st]);
         }
         pdl_wait();  // before this warp writes Y in the epilogue
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
@@ -266,8 +275,9 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
         const uint32_t zrow = smem_u32(zchunk);
         const uint32_t qwarp = smem_u32(smem) + static_cast<uint32_t>(warp * 2048);
         // this lane's shared-memory offsets of its four 16-byte loads per stage:
-        // packed row r = 8 (ss / 2) + 2 t + ss % 2, chunk gq XOR-swizzled by the
-        // row (128-byte TMA swizzle); X' chunk r XOR-swizzled by the token
+        // packed row r = 8 (ss / 2) + 2 t + ss % 2 of the warp's 2 KB slab,
+        // chunk gq XOR-swizzled by the row (128-byte TMA swizzle); X' chunk r
+        // XOR-swizzled by the token
         uint32_t offq[4], offx[4];
 #pragma unroll
         for (int ss = 0; ss < 4; ++ss) {
@@ -281,12 +291,8 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
         for (int a = 0; a < 2; ++a)
 #pragma unroll
             for (int i = 0; i < 4; ++i) R[a][i] = 0.0f;
-        // steps (4 binary16) and zero word of the group(s) this lane finishes
-        // (two named sets rather than an array: a run-time index would put
-        // the array in local memory)
-        uint2 cap_sc0 = make_uint2(0u, 0u), cap_sc1 = cap_sc0;
-        uint32_t cap_z0 = 0u, cap_z1 = 0u;
         bool ok = true;
+        bool meta_ready = false;  // the CTA's steps and zero words have landed
         int st = 0;          // ring slot of the stage
         uint32_t ph = 0;     // its phase parity
         int j = 0;           // group within the batch
@@ -295,16 +301,6 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
             if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph))) {
                 ok = false;
                 break;
-            }
-            const uint8_t *meta = smem + st * kStageBytes + kQStage;
-            if (t == j / kLG) {
-                const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
-                const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
-                const bool second = kLG == 2 && (j & 1);
-                cap_sc0 = second ? cap_sc0 : sc;
-                cap_z0 = second ? cap_z0 : zw;
-                cap_sc1 = second ? sc : cap_sc1;
-                cap_z1 = second ? zw : cap_z1;
             }
             const uint32_t qbase = qwarp + static_cast<uint32_t>(st * kStageBytes);
             const uint32_t xbase = b_group == j ? xrow + static_cast<uint32_t>(it * 256) : zrow;
@@ -339,6 +335,15 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
             if (lane == 0) mbar_arrive(&empty[st]);
 
             if (j == kGPB - 1 || it == ng - 1) {
+                // the steps and zero words (loaded once by the producer) are
+                // first needed here
+                if (!meta_ready) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(meta_bar, 0))) {
+                        ok = false;
+                        break;
+                    }
+                    meta_ready = true;
+                }
                 // batch epilogue: fragment column 2t + u is slot 2t + u = group
                 // g = (2t + u) / MT of the batch, token (2t + u) % MT;
                 // y += step * (R - (1024 S0 + 64 S1) - z (S0 + S1))
@@ -348,11 +353,11 @@ __global__ void __launch_bounds__(32 * (kConsumers + 1), 1)
                     const int slot = 2 * t + u;
                     const int gb = slot / MT;
                     const int tk = slot % MT;
-                    const bool second = kLG == 2 && u == 1;
                     const bool valid = gb <= j;
-                    const float2 gm = valid ? gmeta[tk * ng + base + gb] : make_float2(0.f, 0.f);
-                    const uint2 sc = second ? cap_sc1 : cap_sc0;
-                    const uint32_t zw = second ? cap_z1 : cap_z0;
+                    const int gi = valid ? base + gb : base;
+                    const float2 gm = valid ? gmeta[tk * ng + gi] : make_float2(0.f, 0.f);
+                    const uint2 sc = *reinterpret_cast<const uint2 *>(csteps + gi * 256 + 2 * colw);
+                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(czeros + gi * 64 + 4 * (colw >> 3));
                     const float stp[4] = {__half2float(__ushort_as_half(static_cast<unsigned short>(sc.x & 0xFFFFu))),
                                           __half2float(__ushort_as_half(static_cast<unsigned short>(sc.x >> 16))),
                                           __half2float(__ushort_as_half(static_cast<unsigned short>(sc.y & 0xFFFFu))),
@@ -527,16 +532,17 @@ bool plan_gemv(int M, int K, int N, int num_sms, GemvPlan *pl)
     // (+ 8 B per group half); find the smallest split at or above the choice that fits
     for (; splits <= max_pow2; splits *= 2) {
         const int gmax = (G + splits - 1) / splits;
-        if (static_cast<size_t>(M) * gmax * (256 + 8) <= 80 * 1024) break;
+        if (static_cast<size_t>(M) * gmax * (256 + 8) + static_cast<size_t>(gmax) * 320 <= 80 * 1024) break;
     }
     if (splits > max_pow2) return false;
     pl->splits = splits;
     const int gmax = (G + splits - 1) / splits;
     pl->xpro_bytes = M * gmax * 256;
     pl->gmeta_bytes = (M * gmax * 8 + 15) & ~15;
+    pl->cmeta_bytes = gmax * 320;
     pl->recv_bytes = 8 * kBN * 4;
     pl->smem = 1024 + static_cast<size_t>(pl->stages) * kStageBytes + pl->xpro_bytes + pl->gmeta_bytes +
-               pl->recv_bytes + (2 * pl->stages + 1) * sizeof(uint64_t) + 16 + 256;  // + zero chunk
+               pl->cmeta_bytes + pl->recv_bytes + (2 * pl->stages + 2) * sizeof(uint64_t) + 16 + 256;  // + zero chunk
     return true;
 }
 
@@ -558,6 +564,7 @@ cudaError_t launch_gemv(const GemvPlan &plan, const CUtensorMap &tmQ, const __ha
     prm.splits = plan.splits;
     prm.xpro_bytes = plan.xpro_bytes;
     prm.gmeta_bytes = plan.gmeta_bytes;
+    prm.cmeta_bytes = plan.cmeta_bytes;
     prm.recv_bytes = plan.recv_bytes;
     prm.mask_lo = 0x000F000Fu;
     prm.mask_hi = 0x00F000F0u;
