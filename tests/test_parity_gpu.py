@@ -301,3 +301,18 @@ def test_workspace_counters_return_to_zero():
         torch.cuda.synchronize()
         assert int(ws[:32 * 1024].view(torch.int32).abs().sum().item()) == 0, (K, N, M)
         assert torch.equal(Y1, Y2)
+
+
+def test_chained_calls_are_bit_identical():
+    # Calls chained on one stream overlap under programmatic dependent launch;
+    # every repetition of the same product must give the same bits (a race in
+    # a kernel's rings or reductions shows up here as a few differing columns).
+    ws = torch.zeros(awq.gemm_workspace_size(2, 14336, 28672), dtype=torch.uint8, device="cuda")
+    for (K, N, M, reps) in [(4096, 28672, 1, 24), (4096, 6144, 1, 8), (14336, 4096, 2, 8), (1152, 1032, 1, 8)]:
+        L = synth.make_layer(18, K + N, M=M, K=K, N=N, R=64, device="cuda")
+        s = awq.compute_scales(awq.act_stats(L.Xcal))
+        Q, sc, z = awq.quantize_pack(L.W, s)
+        Ys = [awq.w4a16_gemm(L.X, s, Q, sc, z, workspace=ws) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for i, Y in enumerate(Ys[1:], 1):
+            assert torch.equal(Y, Ys[0]), (K, N, M, i, torch.nonzero(Y != Ys[0])[:4].tolist())
