@@ -226,8 +226,9 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;
+        // boxes of 8 * mt token rows: rows at and beyond M read as zero
         if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
-                       static_cast<uint32_t>(M), CU_TENSOR_MAP_SWIZZLE_128B))
+                       static_cast<uint32_t>(8 * plan.mt), CU_TENSOR_MAP_SWIZZLE_128B))
             return AWQ_ERR_CUDA;
         e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
         if (e != AWQ_OK) return e;

@@ -145,7 +145,8 @@ __global__ void __launch_bounds__(160, 1)
             prefetch_tmap(&tmX);
         }
         pdl_wait();
-        const uint32_t tx = kQStage + 2 * p.M * 128;
+        // the X' boxes hold 8 MT token rows (rows at and beyond M read as zero)
+        const uint32_t tx = kQStage + 2 * (8 * MT) * 128;
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
             const int st = it % S;
@@ -184,10 +185,23 @@ __global__ void __launch_bounds__(160, 1)
         const int t = lane & 3;
         const int colw = 32 * warp + 4 * gq;  // my 4 columns: colw .. colw+3 (tile-local)
         const UnpackConsts uk = p.uk;
+        // this lane's shared-memory offsets within a stage, computed once:
+        // packed row r = 8 (sidx / 2) + 2 t + sidx % 2, chunk gq XOR-swizzled by
+        // the row; X' row of token 8 j + gq, chunk r % 8 XOR-swizzled by the token
+        uint32_t qoff[4], xoff[4][MT];
+#pragma unroll
+        for (int sidx = 0; sidx < 4; ++sidx) {
+            const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);
+            qoff[sidx] = static_cast<uint32_t>(warp * 2048 + r * 128 + ((gq ^ (r & 7)) << 4));
+#pragma unroll
+            for (int j = 0; j < MT; ++j)
+                xoff[sidx][j] = static_cast<uint32_t>(kQStage + (sidx >> 1) * p.xbox + (8 * j + gq) * 128 +
+                                                      (((r & 7) ^ gq) << 4));
+        }
         bool ok = true;
         for (int it = 0; it < ng; ++it) {
             const int st = it % S;
-            if (!mbar_wait(&full[st], (it / S) & 1)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (it / S) & 1))) {
                 ok = false;
                 break;
             }
@@ -206,22 +220,19 @@ __global__ void __launch_bounds__(160, 1)
                 st2[2] = (s23 & 0xFFFFu) * 0x10001u;
                 st2[3] = (s23 >> 16) * 0x10001u;
             }
-            const uint8_t *qslab = stg + warp * 2048;
-            const uint8_t *xstage = stg + kQStage;
+            const uint32_t sbase = smem_u32(stg);
 #pragma unroll
             for (int sidx = 0; sidx < 4; ++sidx) {
-                const int r = 8 * (sidx >> 1) + 2 * t + (sidx & 1);  // packed row in the group
-                const uint4 wq = *reinterpret_cast<const uint4 *>(qslab + r * 128 + ((gq ^ (r & 7)) << 4));
+                uint32_t w[4];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                             : "r"(sbase + qoff[sidx]));
                 uint4 bx[MT];
 #pragma unroll
-                for (int j = 0; j < MT; ++j) {
-                    const int tok = 8 * j + gq;
-                    bx[j] = make_uint4(0u, 0u, 0u, 0u);
-                    if (tok < p.M)
-                        bx[j] = *reinterpret_cast<const uint4 *>(xstage + (sidx >> 1) * p.xbox + tok * 128 +
-                                                                 (((r & 7) ^ (tok & 7)) << 4));
-                }
-                const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+                for (int j = 0; j < MT; ++j)
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(bx[j].x), "=r"(bx[j].y), "=r"(bx[j].z), "=r"(bx[j].w)
+                                 : "r"(sbase + xoff[sidx][j]));
                 uint32_t d[4][4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -329,7 +340,7 @@ cudaError_t configure_one()
 
 int stage_bytes_for(int M)
 {
-    const int xbox = (M * 128 + 1023) & ~1023;
+    const int xbox = (((M + 7) / 8) * 8 * 128 + 1023) & ~1023;
     return (kQStage + 2 * xbox + kMetaBytes + 1023) & ~1023;
 }
 
@@ -405,7 +416,7 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
     prm.N = N;
     prm.G = K / kGroup;
     prm.splits = plan.splits;
-    prm.xbox = (M * 128 + 1023) & ~1023;
+    prm.xbox = (((M + 7) / 8) * 8 * 128 + 1023) & ~1023;
     prm.stage_bytes = stage_bytes_for(M);
     prm.recv_bytes = 8 * plan.mt * kBN * 4;
     prm.uk = unpack_consts();
