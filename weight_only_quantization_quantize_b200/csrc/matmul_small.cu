@@ -350,7 +350,8 @@ cudaError_t configure_small_m()
 {
     const cudaError_t r[] = {configure_one<1, 4>(), configure_one<2, 4>(), configure_one<3, 4>(), configure_one<4, 4>(),
                              configure_one<5, 4>(), configure_one<6, 4>(), configure_one<7, 4>(),
-                             configure_one<8, 4>()};
+                             configure_one<8, 4>(), configure_one<1, 3>(), configure_one<2, 3>(),
+                             configure_one<3, 3>()};
     for (cudaError_t x : r)
         if (x != cudaSuccess) return x;
     return cudaSuccess;
@@ -364,21 +365,29 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
     pl.n_tiles = (N + kBN - 1) / kBN;
     pl.prologue = false;
     pl.kh = 1;
-    // A 4-deep ring for every token count: measured on the 13B set, 8 deep
-    // (fewer resident CTAs) lost 8% at 8 tokens and 30% at 16.
-    pl.stages = 4;
+    // A 4-deep ring, or 3-deep (up to 24 tokens) when that lets more CTAs
+    // share an SM and so a finer split fit in one wave: measured on the 13B
+    // set, resident CTAs beat ring depth (8 deep lost 8% at 8 tokens and 30%
+    // at 16 against 4 deep).
     const int G = K / kGroup;
     int max_pow2 = 1;
     while (max_pow2 * 2 <= 8 && max_pow2 * 2 <= G) max_pow2 *= 2;
     const int stage_bytes = stage_bytes_for(M);
     const int recv_bytes = 8 * pl.mt * kBN * 4;
-    size_t smem = 1024 + static_cast<size_t>(pl.stages) * stage_bytes + recv_bytes + (2 * pl.stages + 1) * 8;
-    const int per_sm = static_cast<int>(228 * 1024 / (smem + 1024));
-    // one wave: the largest power-of-two split with n_tiles * splits <= CTAs resident
-    int splits = 1;
-    while (splits * 2 <= max_pow2 && pl.n_tiles * splits * 2 <= (per_sm < 1 ? 1 : per_sm) * num_sms) splits *= 2;
-    pl.splits = splits;
-    pl.smem = smem;
+    int best_splits = 0;
+    for (int stages = 4; stages >= (pl.mt <= 3 ? 3 : 4); --stages) {
+        const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + recv_bytes + (2 * stages + 1) * 8;
+        const int per_sm = static_cast<int>(228 * 1024 / (smem + 1024));
+        // one wave: the largest power-of-two split with n_tiles * splits <= CTAs resident
+        int splits = 1;
+        while (splits * 2 <= max_pow2 && pl.n_tiles * splits * 2 <= (per_sm < 1 ? 1 : per_sm) * num_sms) splits *= 2;
+        if (splits > best_splits) {
+            best_splits = splits;
+            pl.splits = splits;
+            pl.stages = stages;
+            pl.smem = smem;
+        }
+    }
     return pl;
 }
 
@@ -420,6 +429,14 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
     prm.stage_bytes = stage_bytes_for(M);
     prm.recv_bytes = 8 * plan.mt * kBN * 4;
     prm.uk = unpack_consts();
+    if (plan.stages == 3) {
+        switch (plan.mt) {
+        case 1: return launch_one<1, 3>(plan, tmQ, tmX, prm, st);
+        case 2: return launch_one<2, 3>(plan, tmQ, tmX, prm, st);
+        case 3: return launch_one<3, 3>(plan, tmQ, tmX, prm, st);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     switch (plan.mt) {
     case 1: return launch_one<1, 4>(plan, tmQ, tmX, prm, st);
     case 2: return launch_one<2, 4>(plan, tmQ, tmX, prm, st);
