@@ -179,6 +179,19 @@ def test_matmul_parity_small_shapes(M, K, N):
     assert_y_close(Y, Y32, f"M={M} K={K} N={N} (float oracle)")
 
 
+@pytest.mark.parametrize("M", [1, 8, 20, 40])
+def test_matmul_parity_long_k(M):
+    # k ranges longer than the per-CTA staging of steps and zero words (the
+    # register-fed small-batch kernel then reads them from global memory)
+    K, N = 131072, 64
+    L = synth.make_layer(12, K + M, M=M, K=K, N=N, R=16)
+    s, sr = stats_and_scales_both(L.Xcal)
+    (Q, sc, z), (Qr, scr, zr) = quantize_both(L.W, s.cpu())
+    Y = gemm_gpu(dev(L.X), s, Q, sc, z)
+    Yref = oracle.matmul(h(L.X), sr, Qr, scr, zr, precision=64, nthreads=8)
+    assert_y_close(Y, Yref, f"M={M} K={K} N={N}")
+
+
 def test_matmul_is_deterministic():
     L = synth.make_layer(12, 0, M=1, K=4096, N=4096, R=64)
     s = awq.compute_scales(awq.act_stats(dev(L.Xcal)))

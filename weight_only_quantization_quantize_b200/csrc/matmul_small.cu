@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kBN = 128;            // output columns per CTA
 constexpr int kQStage = 4 * 2048;   // 4 boxes of [16 rows x 32 words]
-constexpr int kMetaBytes = 256 + 64;  // 128 scales + 16 zero words
+constexpr int kMetaGroups = 64;      // the steps and zero words of up to this many groups live in shared memory
 constexpr int kSmemOptIn = 232448;  // 227 KB, the per-block opt-in maximum
 
 
@@ -49,6 +49,8 @@ struct Params {
     int M, K, N, G, splits;
     int xbox;          // bytes reserved per staged X' box
     int stage_bytes;
+    int cmeta_bytes;   // the CTA's steps [group][128] binary16, then zero words [group][16]
+    int meta_smem;     // 1: those are staged in shared memory; 0 (longer k ranges): read from global memory
     int recv_bytes;    // partials pushed to this CTA: [src rank][8 * MT tokens][128 / splits]
     UnpackConsts uk;
 };
@@ -113,17 +115,21 @@ __global__ void __launch_bounds__(160, 1)
 
     pdl_launch_dependents();
 
-    float *recv = reinterpret_cast<float *>(smem + S * p.stage_bytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes + p.recv_bytes);
+    uint8_t *csteps = smem + S * p.stage_bytes;
+    uint8_t *czeros = csteps + ng * 256;
+    float *recv = reinterpret_cast<float *>(csteps + p.cmeta_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(csteps + p.cmeta_bytes + p.recv_bytes);
     uint64_t *empty = full + S;
     uint64_t *recv_bar = empty + S;
+    uint64_t *meta_bar = recv_bar + 1;  // the CTA's steps and zero words have landed
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1 + 32);  // expect_tx arrival + 32 cp.async arrivals
+            mbar_init(&full[i], 1);  // expect_tx arrival
             mbar_init(&empty[i], kConsumers);
         }
         mbar_init(recv_bar, 1);
+        mbar_init(meta_bar, 32);
         fence_barrier_init();
         mbar_arrive_expect_tx(recv_bar, p.M * cpo * p.splits * 4);
     }
@@ -144,6 +150,21 @@ __global__ void __launch_bounds__(160, 1)
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmX);
         }
+        // The steps and zero words of all of the CTA's groups, once (layer
+        // state, so before the wait on the previous kernel).
+        for (int c = lane; p.meta_smem && c < ng * 16; c += 32) {
+            const int gi = c >> 4, c16 = c & 15;
+            const int gg = g_begin + gi;
+            const int n = n0 + 8 * c16;
+            const bool in_s = n < p.N;
+            cp_async_16(csteps + gi * 256 + 16 * c16, p.scales + static_cast<size_t>(gg) * p.N + (in_s ? n : 0),
+                        in_s ? 16u : 0u);
+            const int wi = n0 / 8 + c16;
+            const bool in_z = wi < p.N / 8;
+            cp_async_4(czeros + gi * 64 + 4 * c16, zero_word_src(p.zeros, gg, p.N / 8, in_z ? wi : 0, c16),
+                       in_z ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(meta_bar);
         pdl_wait();
         // the X' boxes hold 8 MT token rows (rows at and beyond M read as zero)
         const uint32_t tx = kQStage + 2 * (8 * MT) * 128;
@@ -164,19 +185,6 @@ __global__ void __launch_bounds__(160, 1)
                 tma_load_2d(stg + kQStage, &tmX, &full[st], g * kGroup, 0);
                 tma_load_2d(stg + kQStage + p.xbox, &tmX, &full[st], g * kGroup + 64, 0);
             }
-            uint8_t *meta = stg + kQStage + 2 * p.xbox;
-            if (lane < 16) {
-                const int n = n0 + 8 * lane;
-                const bool in = n < p.N;
-                cp_async_16(meta + 16 * lane, p.scales + static_cast<size_t>(g) * p.N + (in ? n : 0),
-                            in ? 16u : 0u);
-            } else {
-                const int wi = n0 / 8 + (lane - 16);
-                const bool in = wi < p.N / 8;
-                cp_async_4(meta + 256 + 4 * (lane - 16),
-                           zero_word_src(p.zeros, g, p.N / 8, in ? wi : 0, lane), in ? 4u : 0u);
-            }
-            cp_async_arrive_noinc(&full[st]);
         }
         if (!ok && lane == 0) report(p.status, AWQ_ERR_DEVICE_TIMEOUT);
     } else {
@@ -198,17 +206,29 @@ __global__ void __launch_bounds__(160, 1)
                 xoff[sidx][j] = static_cast<uint32_t>(kQStage + (sidx >> 1) * p.xbox + (8 * j + gq) * 128 +
                                                       (((r & 7) ^ gq) << 4));
         }
-        bool ok = true;
-        for (int it = 0; it < ng; ++it) {
+        bool ok = __all_sync(0xffffffffu, mbar_wait(meta_bar, 0));
+        for (int it = 0; ok && it < ng; ++it) {
             const int st = it % S;
             if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (it / S) & 1))) {
                 ok = false;
                 break;
             }
             const uint8_t *stg = smem + st * p.stage_bytes;
-            const uint8_t *meta = stg + kQStage + 2 * p.xbox;
-            const uint2 sc = *reinterpret_cast<const uint2 *>(meta + 2 * colw);
-            const uint32_t zw = *reinterpret_cast<const uint32_t *>(meta + 256 + 4 * (colw >> 3));
+            uint2 sc;
+            uint32_t zw;
+            if (p.meta_smem) {
+                sc = *reinterpret_cast<const uint2 *>(csteps + it * 256 + 2 * colw);
+                zw = *reinterpret_cast<const uint32_t *>(czeros + it * 64 + 4 * (colw >> 3));
+            } else {
+                // long k ranges: straight from global memory (L2); columns past N read as zero
+                const int g = g_begin + it, n = n0 + colw;
+                const bool in = n < p.N;
+                sc = in ? __ldg(reinterpret_cast<const uint2 *>(p.scales + static_cast<size_t>(g) * p.N + n))
+                        : make_uint2(0u, 0u);
+                zw = !in ? 0u
+                         : (p.zeros ? static_cast<uint32_t>(__ldg(p.zeros + static_cast<size_t>(g) * (p.N / 8) + n / 8))
+                                    : kSymmetricZeroWords[0]);
+            }
             const int zsh = (colw & 7) * 4;
             uint32_t za[4], zb[4], st2[4];
 #pragma unroll
@@ -338,10 +358,18 @@ cudaError_t configure_one()
                                 kSmemOptIn);
 }
 
+// steps (256 B) and zero words (64 B) per group of the largest k range, when
+// they are staged in shared memory
+int cmeta_bytes_for(int G, int splits)
+{
+    const int gmax = (G + splits - 1) / splits;
+    return gmax <= kMetaGroups ? gmax * 320 : 0;
+}
+
 int stage_bytes_for(int M)
 {
     const int xbox = (((M + 7) / 8) * 8 * 128 + 1023) & ~1023;
-    return (kQStage + 2 * xbox + kMetaBytes + 1023) & ~1023;
+    return (kQStage + 2 * xbox + 1023) & ~1023;
 }
 
 }  // namespace
@@ -376,11 +404,21 @@ SmallMPlan plan_small_m(int M, int K, int N, int num_sms)
     const int recv_bytes = 8 * pl.mt * kBN * 4;
     int best_splits = 0;
     for (int stages = 4; stages >= (pl.mt <= 3 ? 3 : 4); --stages) {
-        const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + recv_bytes + (2 * stages + 1) * 8;
-        const int per_sm = static_cast<int>(228 * 1024 / (smem + 1024));
-        // one wave: the largest power-of-two split with n_tiles * splits <= CTAs resident
+        // one wave: the largest power-of-two split with n_tiles * splits <= CTAs
+        // resident (the steps and zero words of a CTA's groups shrink as the
+        // split grows)
         int splits = 1;
-        while (splits * 2 <= max_pow2 && pl.n_tiles * splits * 2 <= (per_sm < 1 ? 1 : per_sm) * num_sms) splits *= 2;
+        size_t smem = 0;
+        for (;;) {
+            const int s2 = splits * 2;
+            const size_t sm2 = 1024 + static_cast<size_t>(stages) * stage_bytes + cmeta_bytes_for(G, s2) + recv_bytes +
+                               (2 * stages + 2) * 8;
+            const int per_sm = static_cast<int>(228 * 1024 / (sm2 + 1024));
+            if (s2 > max_pow2 || pl.n_tiles * s2 > (per_sm < 1 ? 1 : per_sm) * num_sms) break;
+            splits = s2;
+        }
+        smem = 1024 + static_cast<size_t>(stages) * stage_bytes + cmeta_bytes_for(G, splits) + recv_bytes +
+               (2 * stages + 2) * 8;
         if (splits > best_splits) {
             best_splits = splits;
             pl.splits = splits;
@@ -427,6 +465,8 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
     prm.splits = plan.splits;
     prm.xbox = (((M + 7) / 8) * 8 * 128 + 1023) & ~1023;
     prm.stage_bytes = stage_bytes_for(M);
+    prm.cmeta_bytes = cmeta_bytes_for(K / kGroup, plan.splits);
+    prm.meta_smem = prm.cmeta_bytes > 0 ? 1 : 0;
     prm.recv_bytes = 8 * plan.mt * kBN * 4;
     prm.uk = unpack_consts();
     if (plan.stages == 3) {
