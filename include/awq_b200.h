@@ -67,9 +67,11 @@ extern "C" {
 #define AWQ_MAX_K 262144
 #define AWQ_MAX_N 1048576
 #define AWQ_MAX_M 1048576
-#define AWQ_ABI_VERSION 4  /* 2: symmetric weights; 3: 1/s folded upstream;
+#define AWQ_ABI_VERSION 5  /* 2: symmetric weights; 3: 1/s folded upstream;
                                4: every matmul takes a zero-filled workspace;
-                               scale search over alpha; weight clipping */
+                               scale search over alpha; weight clipping;
+                               5: matmul workspaces for M >= 64 hold the
+                               prefill kernel's partial tiles */
 
 typedef enum {
     AWQ_OK = 0,
@@ -214,7 +216,9 @@ AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s
  * never NULL.  It must be zero-filled (e.g. cudaMemsetAsync) before its first
  * use: its first 32 KB are a counter block that a call expects at zero and
  * leaves at zero when it completes without a device error.  The rest holds
- * X / s and is overwritten.  Calls on one stream may share a
+ * X / s and, for M >= 64, the partial sums of output tiles whose k range is
+ * split between CTAs (at most 20 MB); it is overwritten.  The size depends on
+ * M, K and N, not on the device.  Calls on one stream may share a
  * workspace; calls that can run at the same time need separate ones.  After a
  * device error (AWQ_ERR_DEVICE_TIMEOUT) zero the workspace again.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
@@ -314,9 +318,9 @@ AWQ_API awq_status_t awq_scale_search(const uint16_t *xcal, int64_t R, int64_t K
  *
  * Arguments, layouts, tolerance and errors are those of awq_w4a16_gemm, minus
  * the workspace.  Limit: awq_w4a16_gemm_workspace_size(M, K, N) must not exceed
- * AWQ_NOALLOC_SCRATCH_BYTES (32 KB of counters + 2 * M * K bytes of X / s, i.e.
- * M * K <= 2 Mi - 16 Ki elements);
- * larger problems return AWQ_ERR_WORKSPACE before anything runs.
+ * AWQ_NOALLOC_SCRATCH_BYTES (32 KB of counters + 2 * M * K bytes of X / s +
+ * for M >= 64 up to 20 MB of partial tiles; M * K <= 2 Mi - 16 Ki elements
+ * always fits); larger problems return AWQ_ERR_WORKSPACE before anything runs.
  * Set-up: the first call on each device (with that device current) looks up
  * the scratch array's device address; make that first call before any stream
  * capture begins.
@@ -328,7 +332,7 @@ AWQ_API awq_status_t awq_scale_search(const uint16_t *xcal, int64_t R, int64_t K
  * ordering between them) race on the scratch array and give undefined
  * results; order them on one stream or with events.
  */
-#define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+#define AWQ_NOALLOC_SCRATCH_BYTES ((size_t)24 << 20)
 AWQ_API awq_status_t awq_w4a16_gemm_noalloc(const uint16_t *X, const uint16_t *s, const int32_t *Q,
                                             const uint16_t *scales, const int32_t *zeros,
                                             int64_t M, int64_t K, int64_t N, uint16_t *Y,

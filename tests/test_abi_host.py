@@ -52,22 +52,37 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.awq_abi_version() == 4 == awq.ABI_VERSION
+    assert L.awq_abi_version() == 5 == awq.ABI_VERSION
     for code, name in awq.STATUS.items():
         assert awq.status_string(code).startswith(name)
     assert awq.status_string(99) == "AWQ_ERR_UNKNOWN"
 
 
 def test_workspace_sizes(L):
-    # every matmul takes a workspace: 32 KB of arrival counters first, then
-    # X / s (2 M K bytes), then (M <= 2) the decode GEMV's partial sums
+    # every matmul takes a workspace: 32 KB of counters first, then X / s
+    # (2 M K bytes, rounded up to 256), then for M >= 64 the prefill kernel's
+    # fp32 partial tiles: one 128-column slot per CTA, its tokens 128 (M <= 128)
+    # or 256, as many CTAs as the k stages allow at 16 per CTA, at most 20 MB
     counters = 32 * 1024
+
+    def xp(M, K):
+        return (2 * M * K + 255) // 256 * 256
+
+    def partials(M, K, N):
+        bt = 128 if M <= 128 else 256
+        units = -(-N // 128) * -(-M // bt) * (K // 64)
+        ctas = min(max(units // 16, 1), (160 if bt == 256 else 320))
+        return ctas * 128 * bt * 4
+
     g1 = L.awq_w4a16_gemv_workspace_size(4096, 4096)
-    assert g1 == L.awq_w4a16_gemm_workspace_size(1, 4096, 4096)
-    assert g1 >= counters + 2 * 4096
+    assert g1 == L.awq_w4a16_gemm_workspace_size(1, 4096, 4096) == counters + xp(1, 4096)
     assert L.awq_w4a16_gemm_workspace_size(2, 4096, 4096) > g1
-    assert L.awq_w4a16_gemm_workspace_size(48, 5120, 5120) >= counters + 2 * 48 * 5120
-    assert L.awq_w4a16_gemm_workspace_size(4096, 14336, 4096) >= counters + 2 * 4096 * 14336
+    assert L.awq_w4a16_gemm_workspace_size(48, 5120, 5120) == counters + xp(48, 5120)
+    for M, K, N in [(64, 1024, 512), (100, 8192, 264), (128, 128, 8), (129, 4096, 4096), (520, 1152, 1032),
+                    (4096, 14336, 4096), (4096, 4096, 28672)]:
+        assert L.awq_w4a16_gemm_workspace_size(M, K, N) == counters + xp(M, K) + partials(M, K, N), (M, K, N)
+    assert partials(64, 1024, 512) == 4 * 128 * 128 * 4                 # one CTA per tile
+    assert partials(4096, 14336, 4096) == 20 << 20                      # the cap
     assert L.awq_w4a16_gemm_workspace_size(4, 100, 4096) == 0          # invalid shape
     assert L.awq_w4a16_gemv_workspace_size(4096, 4097) == 0            # invalid shape
 

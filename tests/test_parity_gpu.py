@@ -302,10 +302,12 @@ def test_quantize_then_matmul_on_one_stream_without_sync():
 
 
 def test_workspace_counters_return_to_zero():
-    # The decode GEMV counts arrivals on split tiles in the first 32 KB of the
-    # workspace; every call must leave them at zero for the next one.
-    ws = torch.zeros(awq.gemm_workspace_size(2, 14336, 28672), dtype=torch.uint8, device="cuda")
-    for (K, N, M) in [(4096, 6144, 1), (14336, 4096, 2), (1152, 1032, 1), (128, 8, 2), (4096, 28672, 1)]:
+    # The prefill kernel raises flags for split tiles in the first 32 KB of the
+    # workspace; every call must leave that block at zero for the next one.
+    cases = [(4096, 6144, 1), (14336, 4096, 2), (1152, 1032, 1), (128, 8, 2), (4096, 28672, 1),
+             (4096, 6144, 512), (16384, 136, 130), (8192, 264, 100), (1152, 1032, 520)]
+    ws = torch.zeros(max(awq.gemm_workspace_size(M, K, N) for K, N, M in cases), dtype=torch.uint8, device="cuda")
+    for (K, N, M) in cases:
         L = synth.make_layer(16, K + N, M=M, K=K, N=N, R=64, device="cuda")
         s = awq.compute_scales(awq.act_stats(L.Xcal))
         Q, sc, z = awq.quantize_pack(L.W, s)
@@ -320,8 +322,11 @@ def test_chained_calls_are_bit_identical():
     # Calls chained on one stream overlap under programmatic dependent launch;
     # every repetition of the same product must give the same bits (a race in
     # a kernel's rings or reductions shows up here as a few differing columns).
-    ws = torch.zeros(awq.gemm_workspace_size(2, 14336, 28672), dtype=torch.uint8, device="cuda")
-    for (K, N, M, reps) in [(4096, 28672, 1, 24), (4096, 6144, 1, 8), (14336, 4096, 2, 8), (1152, 1032, 1, 8)]:
+    cases = [(4096, 28672, 1, 24), (4096, 6144, 1, 8), (14336, 4096, 2, 8), (1152, 1032, 1, 8),
+             (4096, 6144, 512, 6), (16384, 136, 130, 6)]
+    ws = torch.zeros(max(awq.gemm_workspace_size(M, K, N) for K, N, M, _ in cases), dtype=torch.uint8,
+                     device="cuda")
+    for (K, N, M, reps) in cases:
         L = synth.make_layer(18, K + N, M=M, K=K, N=N, R=64, device="cuda")
         s = awq.compute_scales(awq.act_stats(L.Xcal))
         Q, sc, z = awq.quantize_pack(L.W, s)
@@ -329,3 +334,19 @@ def test_chained_calls_are_bit_identical():
         torch.cuda.synchronize()
         for i, Y in enumerate(Ys[1:], 1):
             assert torch.equal(Y, Ys[0]), (K, N, M, i, torch.nonzero(Y != Ys[0])[:4].tolist())
+
+
+@pytest.mark.parametrize("M,K,N", [(130, 16384, 136), (100, 8192, 264), (64, 4096, 8), (257, 8192, 1032),
+                                   (1000, 4096, 1040)])
+def test_prefill_split_tiles(M, K, N):
+    # Shapes whose one-tile-per-CTA grid would leave most SMs idle run the
+    # stream-K prefill kernel: every CTA takes an equal range of the tiles'
+    # 64-k stages, so a tile's k range is shared by up to 16 CTAs here (long K,
+    # few tiles), with ragged tokens and columns; the CTA holding the tile's
+    # first stages adds the others' partial tiles and writes Y.
+    L = synth.make_layer(21, M + K + N, M=M, K=K, N=N, R=64)
+    s, sr = stats_and_scales_both(L.Xcal)
+    (Q, sc, z), (Qr, scr, zr) = quantize_both(L.W, s.cpu())
+    Y = gemm_gpu(dev(L.X), s, Q, sc, z)
+    Yref = oracle.matmul(h(L.X), sr, Qr, scr, zr, precision=64, nthreads=16)
+    assert_y_close(Y, Yref, f"M={M} K={K} N={N}")

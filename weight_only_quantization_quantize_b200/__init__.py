@@ -41,7 +41,7 @@ LIB_PATH = os.path.join(_PKG, "libawq_b200.so")
 GROUP_SIZE = 128
 W_BIT = 4
 MAX_CALIB_ROWS = 8192
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 STATUS = {
     0: "AWQ_OK", 1: "AWQ_ERR_NULL", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_ALIGN",
@@ -61,7 +61,7 @@ SYMBOLS = (
     "awq_scales_alpha", "awq_scale_search_workspace_size", "awq_scale_search",
     "awq_w4a16_gemm_noalloc",
 )
-NOALLOC_SCRATCH_BYTES = 4 << 20
+NOALLOC_SCRATCH_BYTES = 24 << 20
 
 
 class AwqError(RuntimeError):

@@ -68,7 +68,8 @@ awq_status_t device_ready(int *sms)
                 }
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
-            if (awq::configure_tct() != cudaSuccess || awq::configure_small_m() != cudaSuccess ||
+            if (awq::configure_tct() != cudaSuccess || awq::configure_tsk() != cudaSuccess ||
+                awq::configure_small_m() != cudaSuccess ||
                 awq::configure_gemv() != cudaSuccess || awq::configure_quantize() != cudaSuccess ||
                 awq::configure_tcs() != cudaSuccess || awq::configure_search() != cudaSuccess ||
                 awq::configure_clip() != cudaSuccess) {
@@ -155,18 +156,24 @@ bool matmul_shape_ok(int64_t M, int64_t K, int64_t N)
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace layout of every matmul call:
-//   [0, 32 KB)              a counter block (one uint32 per 128-column tile, up
-//                           to AWQ_MAX_N / 128) reserved for kernels that
-//                           count arrivals on shared tiles; zero between calls
+//   [0, 32 KB)              a counter block (AWQ_MAX_N / 128 uint32 words) for
+//                           kernels that signal between CTAs (the stream-K
+//                           prefill kernel's partial-tile flags); zero between calls
 //   [32 KB, +2MK)           X / s (binary16, pair-permuted) for the small-batch
 //                           and tcgen05 paths
+//   then, for M >= 64       the stream-K prefill kernel's fp32 partial tiles
+//                           (one per CTA whose k range starts inside a tile)
 constexpr size_t kCounterBytes = static_cast<size_t>(AWQ_MAX_N / 128) * sizeof(uint32_t);
+constexpr int64_t kPrefillMinM = 64;  // from here on the prefill kernel runs
 
 size_t xp_bytes(int64_t M, int64_t K) { return round_up(static_cast<size_t>(2 * M * K), 256); }
 
-size_t workspace_bytes(int64_t M, int64_t K)
+size_t workspace_bytes(int64_t M, int64_t K, int64_t N)
 {
-    return kCounterBytes + xp_bytes(M, K);
+    size_t b = kCounterBytes + xp_bytes(M, K);
+    if (M >= kPrefillMinM)
+        b += awq::tsk_partial_bytes(static_cast<int>(M), static_cast<int>(K), static_cast<int>(N));
+    return b;
 }
 
 awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
@@ -181,7 +188,7 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         (zeros && !aligned16(zeros)) || !aligned16(Y) || (ws && !aligned16(ws)) ||
         (dev_status && !aligned4(dev_status)))
         return AWQ_ERR_ALIGN;
-    if (ws == nullptr || ws_bytes < workspace_bytes(M, K)) return AWQ_ERR_WORKSPACE;
+    if (ws == nullptr || ws_bytes < workspace_bytes(M, K, N)) return AWQ_ERR_WORKSPACE;
     int sms = 0;
     awq_status_t e = device_ready(&sms);
     if (e != AWQ_OK) return e;
@@ -210,7 +217,7 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
     // mma.sync gives: tcgen05 with the dequantized weights in tensor memory as
     // the 128-row operand (measured on the 13B shapes: as fast at 24 tokens,
     // faster from 32, slower at 8 and 16).
-    if (M >= 24 && M < 64) {
+    if (M >= 24 && M < kPrefillMinM) {
         const awq::TcsPlan plan = awq::plan_tcs(m, k, n, sms);
         if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
                        static_cast<uint32_t>(plan.nt), CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -221,7 +228,7 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         if (e != AWQ_OK) return e;
         return from_cuda(awq::launch_tcs(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
     }
-    if (M < 64) {
+    if (M < kPrefillMinM) {
         const awq::SmallMPlan plan = awq::plan_small_m(m, k, n, sms);
         if (!encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 32, 16,
                        CU_TENSOR_MAP_SWIZZLE_128B))
@@ -235,15 +242,23 @@ awq_status_t run_matmul(const uint16_t *X, const uint16_t *s, const int32_t *Q,
         return from_cuda(awq::launch_small_m(plan, tmQ, tmX, hX, hs, hsc, zeros, hY, m, k, n,
                                              dev_status, st));
     }
+    // One tile per CTA, or stream-K over the tiles' k stages where that grid
+    // would leave SMs idle (few tiles, or a last wave that fills few SMs).
     const awq::TctPlan plan = awq::plan_tct(m, k, n, sms);
+    const awq::TskPlan skplan = awq::plan_tsk(m, k, n, sms);
+    const bool sk = awq::tsk_preferred(plan, skplan, k, sms);
     if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xp, K, M, K * 2, 64,
-                   static_cast<uint32_t>(plan.bt), CU_TENSOR_MAP_SWIZZLE_128B) ||
+                   static_cast<uint32_t>(sk ? skplan.bt : plan.bt), CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_INT32, Q, N, K / 8, N * 4, 128, 8,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
         return AWQ_ERR_CUDA;
     e = from_cuda(awq::launch_prescale(hX, hs, m, k, Xp, st));
     if (e != AWQ_OK) return e;
-    return from_cuda(awq::launch_tct(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
+    if (!sk) return from_cuda(awq::launch_tct(plan, tmX, tmQ, hsc, zeros, hY, m, k, n, dev_status, st));
+    float *partials = reinterpret_cast<float *>(wsb + kCounterBytes + xp_bytes(M, K));
+    uint32_t *flags = reinterpret_cast<uint32_t *>(wsb);
+    return from_cuda(
+        awq::launch_tsk(skplan, tmX, tmQ, hsc, zeros, hY, m, k, n, partials, flags, dev_status, st));
 }
 
 }  // namespace
@@ -404,7 +419,7 @@ awq_status_t awq_fold_inverse_scale(const uint16_t *a, int64_t rows, int64_t K, 
 
 size_t awq_w4a16_gemv_workspace_size(int64_t K, int64_t N)
 {
-    return matmul_shape_ok(1, K, N) ? workspace_bytes(1, K) : 0;
+    return matmul_shape_ok(1, K, N) ? workspace_bytes(1, K, N) : 0;
 }
 
 awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t *Q,
@@ -418,7 +433,7 @@ awq_status_t awq_w4a16_gemv(const uint16_t *X, const uint16_t *s, const int32_t 
 
 size_t awq_w4a16_gemm_workspace_size(int64_t M, int64_t K, int64_t N)
 {
-    return matmul_shape_ok(M, K, N) ? workspace_bytes(M, K) : 0;
+    return matmul_shape_ok(M, K, N) ? workspace_bytes(M, K, N) : 0;
 }
 
 awq_status_t awq_w4a16_gemm(const uint16_t *X, const uint16_t *s, const int32_t *Q,
@@ -442,7 +457,7 @@ enum { kSmm, kSm, kSs, kSQ, kSsc, kSz, kSWT, kSYr, kSYq, kSpart, kSparts };
 void search_layout(int64_t R, int64_t K, int64_t N, size_t off[kSparts + 1])
 {
     const size_t G = static_cast<size_t>(K / kGroup);
-    const size_t sz[kSparts] = {workspace_bytes(R, K),
+    const size_t sz[kSparts] = {workspace_bytes(R, K, N),
                                 4 * static_cast<size_t>(K),
                                 2 * static_cast<size_t>(K),
                                 4 * static_cast<size_t>(K / 8) * N,

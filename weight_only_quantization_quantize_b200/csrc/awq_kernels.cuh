@@ -56,7 +56,7 @@ cudaError_t launch_small_m(const SmallMPlan &plan, const CUtensorMap &tmQ, const
                            int32_t *status, cudaStream_t st);
 
 // matmul_tct.cu -- M >= 64: tcgen05 with the dequantized weights in TMEM
-// (transposed tile: 128 output columns x bt tokens)
+// (transposed tile: 128 output columns x bt tokens), one tile per CTA
 struct TctPlan {
     int bt;        // tokens per tile: 128 or 256
     int m_tiles, n_tiles;
@@ -67,6 +67,27 @@ cudaError_t configure_tct();
 cudaError_t launch_tct(const TctPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
                        const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
                        int32_t *status, cudaStream_t st);
+
+// matmul_tsk.cu -- the same tile split along K by stream-K, for grids that
+// one tile per CTA would leave partly idle
+struct TskPlan {
+    int bt;        // tokens per tile: 128 or 256
+    int m_tiles, n_tiles;
+    int grid;      // CTAs, each a contiguous range of the tiles' 64-k stages
+    size_t smem;
+};
+TskPlan plan_tsk(int M, int K, int N, int num_sms);
+// True when the stream-K grid is expected to finish before the one-tile-per-CTA grid.
+bool tsk_preferred(const TctPlan &dp, const TskPlan &sk, int K, int num_sms);
+// Workspace bytes for the partial tiles (one slot per CTA of the largest grid
+// any device gets for this problem).
+size_t tsk_partial_bytes(int M, int K, int N);
+cudaError_t configure_tsk();
+// partials: tsk_partial_bytes(M, K, N) bytes; flags: 8 zero words per CTA,
+// left at zero by a call that completes without a device error.
+cudaError_t launch_tsk(const TskPlan &plan, const CUtensorMap &tmX, const CUtensorMap &tmQ,
+                       const __half *scales, const int32_t *zeros, __half *Y, int M, int K, int N,
+                       float *partials, uint32_t *flags, int32_t *status, cudaStream_t st);
 
 // matmul_tcs.cu -- 24 <= M < 64: tcgen05 with the weights as the 128-row operand in TMEM
 struct TcsPlan {
