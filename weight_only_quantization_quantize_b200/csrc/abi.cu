@@ -4,7 +4,7 @@
 // one-time per-device architecture check, TMA descriptor encoding, workspace
 // accounting and the choice of tile path.  Every step of the computation runs
 // in the kernels of quantize.cu, fold.cu, gemv.cu, matmul_small.cu,
-// matmul_tcs.cu and matmul_tct.cu.
+// matmul_tcs.cu, matmul_tct.cu, matmul_tsk.cu, search.cu and clip.cu.
 #include <mutex>
 
 #include "awq_kernels.cuh"
