@@ -222,7 +222,11 @@ AWQ_API awq_status_t awq_quantize_pack_clip(const uint16_t *W, const uint16_t *s
  * workspace; calls that can run at the same time need separate ones.  After a
  * device error (AWQ_ERR_DEVICE_TIMEOUT) zero the workspace again.
  * Device errors: AWQ_ERR_DEVICE_TIMEOUT if an internal pipeline wait ran out
- * (Y is then unspecified).
+ * (Y is then unspecified).  For M >= 64 with few output tiles the call may run
+ * a grid whose CTAs wait (up to 1 s) for partial sums from later CTAs of the
+ * same grid; the grid is sized so that all of its CTAs fit on the GPU at once,
+ * so a kernel on another stream that keeps SMs occupied for longer than that
+ * can make such a call report AWQ_ERR_DEVICE_TIMEOUT instead of finishing.
  * Stream ordering: these kernels use programmatic dependent launch, so a call
  * may start while the previous kernel on the stream is still finishing.  X and
  * the workspace are touched only after that kernel has completed.  Q, scales
