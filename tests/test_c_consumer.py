@@ -50,7 +50,8 @@ def _compiler(name):
 
 
 def test_plain_c_program_links_and_calls_the_library(tmp_path):
-    awq.lib()  # the library has been built
+    from weight_only_quantization_quantize_b200 import _build
+    _build.build()  # in-tree, if it is not built yet
     src = tmp_path / "consumer.c"
     exe = tmp_path / "consumer"
     src.write_text(C_PROGRAM)
